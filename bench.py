@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the LVSA sparse-attention hot path on B200.
+
+One step = the whole per-denoising-step path for one synthetic batch:
+build the frame lists of step s on the host (C ABI), upload them (pinned
+memory, async on the stream), run the sm_100a sparse-attention kernel.  The
+timed region holds exactly K steps (s = W..W+K-1 after W warm-up steps),
+bracketed by a barrier and device synchronisation, timed with CUDA events on
+the launching stream; for N > 1 the max over ranks is taken.  Inputs (Q, K, V,
+O = 2.3 GB for the Wan-1.3B 6x workload) are larger than the 126 MB L2, so no
+flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl lvsa|reference]
+
+Prints one JSON line on rank 0.  ``--impl reference`` times the fp64 CPU
+oracle (a bounded sample of the same workload per step) on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn ms/call & effective TFLOP/s, T=121×1560 tok, 12 heads, d=128"
+DEFAULT_WORKLOAD = "wan1.3b_6x"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops_per_call(w) -> float:
+    """Selected blocks only: QK^T and PV, 2*P*(L*P)*d flops each per (b, h, t)."""
+    return 4.0 * w.B * w.H * w.T * w.L * w.P * w.P * w.d
+
+
+def algorithmic_bytes(w) -> float:
+    """Q, K, V read once and O written once, bf16."""
+    return 4.0 * w.B * w.T * w.P * w.H * w.d * 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            sel = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "200"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        power = [r[2] for r in rows]
+        busy = [r for r in rows if r[2] > 0.5 * max(power)] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i, v in enumerate(r[3][1:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in busy), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(power), "samples": len(rows), "samples_under_load": len(busy),
+                "reasons": reasons}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def cpu_oracle_sample(w, seconds: float, seed: int = 0):
+    """Time the fp64 oracle on whole (head, query-frame) units of the workload
+    until ``seconds`` of CPU work are done.  Returns (flops, elapsed, units)."""
+    import numpy as np
+    import torch
+
+    from block_sparse_attention_frame_b200 import synthetic
+    from oracle import attention as OA
+    from oracle import lists as OL
+
+    # the sample needs the K/V tokens of the frames it touches only; draw the
+    # workload's tensors on the CPU with a smaller head count to bound memory
+    sub = synthetic.Workload(w.name + "-cpu-sample", T=w.T, P=w.P, H=1, d=w.d, C=w.C, W=w.W, seed=w.seed + 17)
+    q, k, v = synthetic.make_qkv(sub, device="cpu")
+    lists = OL.frame_lists(w.T, w.C, w.W, 0)
+    g = np.random.default_rng(seed)
+    frames = list(g.permutation(w.T))
+    done = 0
+    flops = 0.0
+    t0 = time.perf_counter()
+    for t in frames:
+        rows = range(int(t) * w.P, (int(t) + 1) * w.P)
+        OA.sparse_attention_rows(q, k, v, lists, w.P, rows)
+        done += 1
+        flops += 4.0 * w.P * (len(lists[int(t)]) * w.P) * w.d
+        if time.perf_counter() - t0 >= seconds:
+            break
+    return flops, time.perf_counter() - t0, done
+
+
+def host_threads() -> int:
+    try:
+        import threadpoolctl
+
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, on the host cores: each step one bounded sample."""
+    from block_sparse_attention_frame_b200 import synthetic
+
+    if rank != 0:
+        return 0
+    w = synthetic.WORKLOADS[args.workload]
+    per_step = args.ref_seconds or max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, per_step * 0.25)
+    tot_f, tot_t, units = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        f, t, u = cpu_oracle_sample(w, per_step)
+        tot_f += f
+        tot_t += t
+        units += u
+    value = tot_f / tot_t / 1e12
+    ms_call = flops_per_call(w) / (value * 1e12) * 1e3
+    sample = (f"{units} (head, query frame) units of {w.P} query rows each over {args.steps} steps "
+              f"(~{per_step:.1f} s per step), extrapolated to the full call")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, world):
+    return {"workload": w.name, "T": w.T, "tokens_per_frame": w.P, "heads": w.H, "head_dim": w.d, "C": w.C,
+            "W": w.W, "G": max(0, w.C - w.W) if w.C < w.T else 0, "global_batch": w.B * world,
+            "seq_len": w.T * w.P, "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2 (Q+K+V+O working set "
+                  f"{algorithmic_bytes(w) / 1e9:.2f} GB vs 126 MB), no flush"}
+
+
+def run_lvsa(args, rank, world, local):
+    import numpy as np
+    import torch
+
+    import block_sparse_attention_frame_b200 as lvsa
+    from block_sparse_attention_frame_b200 import synthetic
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = synthetic.WORKLOADS[args.workload]
+    F = flops_per_call(w)
+    q, k, v = synthetic.make_qkv(w, device=dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    nsteps = args.warmup + args.steps
+    # per-step pinned host list buffers (the host writes step s+1 while step s copies)
+    pinned = [torch.empty((w.T, w.L), dtype=torch.int32).pin_memory() for _ in range(nsteps)]
+    lists_dev = torch.empty((w.T, w.L), dtype=torch.int32, device=dev)
+    build_us = []
+
+    def step(s, host_list_buf):
+        t0 = time.perf_counter()
+        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=host_list_buf.numpy())
+        build_us.append((time.perf_counter() - t0) * 1e6)
+        lists_dev.copy_(host_list_buf, non_blocking=True)
+        lvsa.lvsa_attention(q, k, v, lists_dev, w.P, out=out, stream=stream)
+
+    # ---------------------------------------------------------------- device-resident timing
+    for s in range(args.warmup):
+        step(s, pinned[s])
+    torch.cuda.synchronize()
+    build_us.clear()
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            s = args.warmup + i
+            t0 = time.perf_counter()
+            lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=pinned[s].numpy())
+            build_us.append((time.perf_counter() - t0) * 1e6)
+            lists_dev.copy_(pinned[s], non_blocking=True)
+            ev_k[i][0].record(stream)
+            lvsa.lvsa_attention(q, k, v, lists_dev, w.P, out=out, stream=stream)
+            ev_k[i][1].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
+    kernel_ms = [a.elapsed_time(b) for a, b in ev_k]
+    status = lvsa.lvsa_get_device_status(clear=True)
+    if status:
+        raise RuntimeError(f"device status {status:#x} after the timed region")
+    ms_per_step = elapsed_ms / args.steps
+    value = world * F * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    # ---------------------------------------------------------------- dense control (same kernel, C = T)
+    dense_lists = torch.from_numpy(lvsa.lvsa_build_frame_lists(w.T, w.T, 1, 0)).to(dev)
+    dout = torch.empty_like(q)
+    lvsa.lvsa_attention(q, k, v, dense_lists, w.P, out=dout)
+    torch.cuda.synchronize()
+    dense_calls = 2
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(dense_calls):
+        lvsa.lvsa_attention(q, k, v, dense_lists, w.P, out=dout)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = d0.elapsed_time(d1) / dense_calls
+    del dout
+
+    # ---------------------------------------------------------------- end to end with host buffers
+    qh = q.cpu().pin_memory()
+    kh = k.cpu().pin_memory()
+    vh = v.cpu().pin_memory()
+    oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step(s):
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=pinned[s % nsteps].numpy())
+        lists_dev.copy_(pinned[s % nsteps], non_blocking=True)
+        lvsa.lvsa_attention(q, k, v, lists_dev, w.P, out=out, stream=stream)
+        oh.copy_(out, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = 3 * q.numel() * q.element_size() + w.T * w.L * 4
+    d2h = out.numel() * out.element_size()
+
+    # ---------------------------------------------------------------- roofline of the kernel
+    peaks, peak_src = load_peaks()
+    kern_avg_ms = sum(kernel_ms) / len(kernel_ms)
+    achieved = F / (kern_avg_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            with open(tpath) as f:
+                tj = json.load(f)
+            if tj.get("workload") == w.name and tj.get("kernel_source_hash") == kernel_source_hash():
+                traffic = tj.get("bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w, world),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                     "kernel_ms_avg": kern_avg_ms, "flops_per_launch": F},
+        "e2e": {"value": F / (e2e_ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "dense_control": {"ms_per_call": dense_ms, "tflops": flops_per_call_dense(w) / (dense_ms * 1e-3) / 1e12,
+                          "speedup_sparse_vs_dense": dense_ms / kern_avg_ms},
+        "list_build_us": {"median": statistics.median(build_us), "max": max(build_us)},
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, t, units = cpu_oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
+                                "sample": f"{units} (head, query frame) units of {w.P} rows, "
+                                          f"{t:.1f} s of fp64 numpy on the host"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def flops_per_call_dense(w) -> float:
+    return 4.0 * w.B * w.H * w.T * w.T * w.P * w.P * w.d
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in ("block_sparse_attention_frame_b200/csrc/attention.cu", "block_sparse_attention_frame_b200/csrc/sm100.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="lvsa", choices=["lvsa", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=0.0, help="reference arm: CPU seconds per step")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps; the JSON reports the count used
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, rank, world)
+        return run_lvsa(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

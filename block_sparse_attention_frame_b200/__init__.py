@@ -1,0 +1,183 @@
+"""Python binding of the LVSA B200 library (``liblvsa.so``).
+
+Argument marshalling only: every step of the path runs in the C++/CUDA
+library.  PyTorch supplies device memory and streams.  If the library is not
+built this module raises on import; there is no CPU or PyTorch fallback.
+
+Functions carry the C ABI's names (declared in ``include/lvsa.h``):
+
+``lvsa_build_frame_lists(T, C, W, step)`` -> int32 numpy array [T, min(C,T)]
+``lvsa_build_anchors(T, C, W, step)``     -> int32 numpy array [G]
+``lvsa_attention(q, k, v, lists, tokens_per_frame, scale=0, out=None, stream=None)``
+``lvsa_get_device_status(clear=False)``   -> int (LVSA_DEV_* bits)
+``lvsa_set_wait_budget_ns(ns)``, ``lvsa_watchdog_selftest(budget_ns, stream=None)``
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblvsa.so")
+
+LVSA_OK = 0
+LVSA_ERR_INVALID_ARG = 1
+LVSA_ERR_UNSUPPORTED = 2
+LVSA_ERR_CUDA = 3
+LVSA_ERR_TIMEOUT = 4
+LVSA_ERR_BUFFER_TOO_SMALL = 5
+LVSA_ERR_BAD_LIST = 6
+LVSA_DEV_TIMEOUT = 0x1
+LVSA_DEV_BAD_LIST = 0x2
+
+EXPORTED = [
+    "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_get_device_status",
+    "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_status_string", "lvsa_version",
+]
+
+
+class LvsaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_frame_b200.build` "
+        "(there is no fallback path)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_c_int, _c_size, _c_ll, _c_ull, _c_float, _c_vp = (ctypes.c_int, ctypes.c_size_t, ctypes.c_longlong,
+                                                     ctypes.c_ulonglong, ctypes.c_float, ctypes.c_void_p)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+
+_lib.lvsa_build_frame_lists.argtypes = [_c_int, _c_int, _c_int, _c_ll, _i32p, _c_size, ctypes.POINTER(_c_int)]
+_lib.lvsa_build_frame_lists.restype = _c_int
+_lib.lvsa_build_anchors.argtypes = [_c_int, _c_int, _c_int, _c_ll, _i32p, _c_size, ctypes.POINTER(_c_int)]
+_lib.lvsa_build_anchors.restype = _c_int
+_lib.lvsa_attention.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                _c_float, _c_vp, _c_vp]
+_lib.lvsa_attention.restype = _c_int
+_lib.lvsa_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), _c_int]
+_lib.lvsa_get_device_status.restype = _c_int
+_lib.lvsa_set_wait_budget_ns.argtypes = [_c_ull]
+_lib.lvsa_set_wait_budget_ns.restype = _c_int
+_lib.lvsa_watchdog_selftest.argtypes = [_c_ull, _c_vp]
+_lib.lvsa_watchdog_selftest.restype = _c_int
+_lib.lvsa_status_string.argtypes = [_c_int]
+_lib.lvsa_status_string.restype = ctypes.c_char_p
+_lib.lvsa_version.argtypes = []
+_lib.lvsa_version.restype = _c_int
+
+
+def status_string(status: int) -> str:
+    return _lib.lvsa_status_string(int(status)).decode()
+
+
+lvsa_status_string = status_string
+
+
+def lvsa_version() -> int:
+    return int(_lib.lvsa_version())
+
+
+def _check(fn: str, st: int) -> None:
+    if st != LVSA_OK:
+        raise LvsaError(fn, st)
+
+
+def lvsa_build_frame_lists(T: int, C: int, W: int, step: int, out: np.ndarray | None = None) -> np.ndarray:
+    """Frame lists A(t) of step ``step`` as int32 [T, min(C, T)] (host)."""
+    L = ctypes.c_int(0)
+    if out is None:
+        st = _lib.lvsa_build_frame_lists(T, C, W, step, None, 0, ctypes.byref(L))
+        if st not in (LVSA_OK, LVSA_ERR_BUFFER_TOO_SMALL):
+            _check("lvsa_build_frame_lists", st)
+        out = np.empty((T, L.value), dtype=np.int32)
+    if out.dtype != np.int32 or not out.flags.c_contiguous:
+        raise ValueError("out must be a C-contiguous int32 array")
+    st = _lib.lvsa_build_frame_lists(T, C, W, step, out.ctypes.data_as(_i32p), out.size, ctypes.byref(L))
+    _check("lvsa_build_frame_lists", st)
+    return out.reshape(T, L.value)
+
+
+def lvsa_build_anchors(T: int, C: int, W: int, step: int) -> np.ndarray:
+    """Anchor frames G_s of step ``step`` as int32 [G] (host)."""
+    G = ctypes.c_int(0)
+    st = _lib.lvsa_build_anchors(T, C, W, step, None, 0, ctypes.byref(G))
+    if st not in (LVSA_OK, LVSA_ERR_BUFFER_TOO_SMALL):
+        _check("lvsa_build_anchors", st)
+    out = np.empty(G.value, dtype=np.int32)
+    if G.value:
+        _check("lvsa_build_anchors",
+               _lib.lvsa_build_anchors(T, C, W, step, out.ctypes.data_as(_i32p), out.size, ctypes.byref(G)))
+    return out
+
+
+def _stream_ptr(stream, device):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def lvsa_attention(q, k, v, lists, tokens_per_frame: int, scale: float = 0.0, out=None, stream=None):
+    """Block-sparse attention on the GPU.
+
+    q, k, v: CUDA bf16 tensors [batch, T*tokens_per_frame, heads, d], contiguous.
+    lists:   CUDA int32 tensor [T, L] of frame indices.
+    Returns ``out`` (allocated with torch if not given).  Asynchronous on ``stream``
+    (default: the current torch stream of q's device).
+    """
+    import torch
+
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(x, torch.Tensor) or x.device.type != "cuda" or x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+        if not x.is_contiguous() or x.dim() != 4 or x.shape != q.shape:
+            raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q")
+    if lists.device.type != "cuda" or lists.dtype != torch.int32 or lists.dim() != 2 or not lists.is_contiguous():
+        raise TypeError("lists must be a contiguous CUDA int32 tensor [T, L]")
+    B, ntok, H, d = q.shape
+    T, L = lists.shape
+    if ntok != T * tokens_per_frame:
+        raise ValueError(f"q has {ntok} tokens, expected T*tokens_per_frame = {T * tokens_per_frame}")
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device != q.device:
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q on q's device")
+    with torch.cuda.device(q.device):
+        st = _lib.lvsa_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), lists.data_ptr(), L, T,
+                                 tokens_per_frame, H, d, B, float(scale), out.data_ptr(),
+                                 _stream_ptr(stream, q.device))
+    _check("lvsa_attention", st)
+    return out
+
+
+def lvsa_attention_raw(q_ptr: int, k_ptr: int, v_ptr: int, lists_ptr: int, L: int, T: int, P: int, H: int,
+                       d: int, B: int, scale: float, out_ptr: int, stream_ptr: int) -> int:
+    """The C call with raw device pointers; returns the status code unchanged."""
+    return int(_lib.lvsa_attention(q_ptr, k_ptr, v_ptr, lists_ptr, L, T, P, H, d, B, float(scale), out_ptr,
+                                   ctypes.c_void_p(stream_ptr)))
+
+
+def lvsa_get_device_status(clear: bool = False) -> int:
+    flags = ctypes.c_uint(0)
+    _check("lvsa_get_device_status", _lib.lvsa_get_device_status(ctypes.byref(flags), 1 if clear else 0))
+    return int(flags.value)
+
+
+def lvsa_set_wait_budget_ns(ns: int) -> None:
+    _check("lvsa_set_wait_budget_ns", _lib.lvsa_set_wait_budget_ns(int(ns)))
+
+
+def lvsa_watchdog_selftest(budget_ns: int, stream=None) -> None:
+    import torch
+
+    _check("lvsa_watchdog_selftest",
+           _lib.lvsa_watchdog_selftest(int(budget_ns), _stream_ptr(stream, torch.cuda.current_device())))

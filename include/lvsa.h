@@ -1,0 +1,157 @@
+/*
+ * lvsa.h -- C ABI of the B200 (sm_100a) library for LVSA frame-granular
+ * block-sparse self-attention.
+ *
+ * Method: "LVSA: Training-Free Sparse Attention for Long Video Diffusion".
+ * A query frame t of a video of T latent frames attends only to the frames of
+ *     A(t) = G_s U W(t)
+ * (gist.science technical summary, section 2 "Core Mechanism"): G_s are
+ * G = C - W global anchor frames whose offset rotates with the denoising step
+ * s, W(t) is a local window of W frames that is extended until |A(t)| reaches
+ * the budget C (same summary, "Rotating Global Anchors" and "Expanded Adaptive
+ * Windows"; techwalker article "华为巴黎研究院让AI视频“不再原地打转”", sections
+ * 二 and 三).
+ *
+ * Conventions for every entry point:
+ *  - Every function returns an lvsa_status; nothing is thrown, nothing aborts.
+ *  - Arguments are validated before any CUDA call or launch; on an error return
+ *    no output has been written and nothing was launched.
+ *  - The library never allocates device memory and never frees caller memory:
+ *    the caller owns every buffer it passes.
+ *  - Thread safety: lvsa_build_frame_lists is pure; lvsa_attention may be called
+ *    from several host threads on different streams.
+ */
+#ifndef LVSA_H
+#define LVSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LVSA_OK = 0,
+  LVSA_ERR_INVALID_ARG = 1,      /* a size, pointer or parameter is out of range */
+  LVSA_ERR_UNSUPPORTED = 2,      /* valid but not supported here (e.g. head dim not 64/128, no sm_100 device) */
+  LVSA_ERR_CUDA = 3,             /* a CUDA runtime/driver call failed */
+  LVSA_ERR_TIMEOUT = 4,          /* a device-side bounded wait ran out (see lvsa_get_device_status) */
+  LVSA_ERR_BUFFER_TOO_SMALL = 5, /* the output capacity is below what the call must write */
+  LVSA_ERR_BAD_LIST = 6          /* a device frame list held an entry outside [0, T) */
+} lvsa_status;
+
+/* Device status bits reported by lvsa_get_device_status. */
+#define LVSA_DEV_TIMEOUT  0x1u   /* a kernel's bounded wait expired; that CTA stopped early */
+#define LVSA_DEV_BAD_LIST 0x2u   /* a frame-list entry was outside [0, T); the entry was skipped */
+
+/*
+ * lvsa_build_frame_lists -- per-query-frame KV frame lists A(t) for step `step`.
+ *
+ * Defines: A(t) = G_s U W(t) (gist.science summary, section 2 "Core
+ * Mechanism"), with
+ *   - G = C - W anchors at spacing about T / (C - W) (techwalker article,
+ *     section 二), placed at floor(k*T/G), k = 0..G-1, shifted by step mod T
+ *     (same article, section 三: one frame per step, modulo the total frame
+ *     count);
+ *   - the window of W frames centred on t (lo = t - W/2), shifted inward at the
+ *     sequence ends;
+ *   - extension (gist.science summary, "Expanded Adaptive Windows"; techwalker
+ *     article, section 二): new non-anchor frames are added alternately right
+ *     then left of the window until |A(t)| = C; a side at the sequence end is
+ *     skipped;
+ *   - C >= T: every row is 0..T-1 (dense attention).
+ *
+ * Arguments:
+ *   T, C, W  latent frames, frame budget, window size; need T >= 1, 1 <= W <= C.
+ *   step     denoising step, >= 0.
+ *   out      HOST int32 buffer, caller-owned, row-major [T][L] with
+ *            L = min(C, T); each row strictly ascending frame indices in [0,T).
+ *   out_capacity  number of int32 elements `out` can hold (>= T*L).
+ *   out_L    optional (may be NULL): receives L.
+ * Errors: LVSA_ERR_INVALID_ARG (parameters), LVSA_ERR_BUFFER_TOO_SMALL (capacity;
+ *   *out_L is still set so the caller can size the buffer; out may be NULL then).
+ * Host only; no CUDA call; cost O(T*C).
+ */
+lvsa_status lvsa_build_frame_lists(int T, int C, int W, long long step,
+                                   int32_t* out, size_t out_capacity, int* out_L);
+
+/*
+ * lvsa_build_anchors -- the G = C - W anchor frames of step `step`, ascending
+ * (techwalker article, section 三; gist.science summary, "Rotating Global
+ * Anchors").  out: HOST int32 buffer of out_capacity elements (>= G).
+ * *out_G receives G (0 when C >= T or W == C: no anchors).
+ * Errors as lvsa_build_frame_lists.
+ */
+lvsa_status lvsa_build_anchors(int T, int C, int W, long long step,
+                               int32_t* out, size_t out_capacity, int* out_G);
+
+/*
+ * lvsa_attention -- frame-granular block-sparse softmax attention.
+ *
+ * Defines (gist.science summary, section 2 "Core Mechanism" and "Complexity";
+ * page 1 "LVSA hoạt động như thế nào": block-sparse attention over structured
+ * windows plus rotating anchors): for query token i of frame t, batch b, head h
+ *     out[b,i,h,:] = sum_j softmax_j(scale * q[b,i,h,:] . k[b,j,h,:]) v[b,j,h,:]
+ * with j running over the tokens of the frames listed in lists[t][0..L-1],
+ * one softmax over all of them together.  Cost O(T * L * P^2 * d) per head.
+ *
+ * Arguments:
+ *   q, k, v  DEVICE bf16, contiguous [batch][T*tokens_per_frame][heads][d]
+ *            (frame-major tokens: token t*P + i is patch i of frame t), 16-byte
+ *            aligned.  Values must be finite.
+ *   lists    DEVICE int32 [T][L], row t = the frames attended by query frame t
+ *            (as written by lvsa_build_frame_lists, or 0..T-1 in every row for
+ *            dense attention).  Rows should be ascending without duplicates:
+ *            runs of consecutive frames are fetched as one token range, a
+ *            duplicated frame is attended twice.  Entries outside [0,T) are
+ *            skipped and flag LVSA_DEV_BAD_LIST.
+ *   L        list width, 1 <= L <= T.
+ *   T, tokens_per_frame (P), heads (H), d, batch: sizes; d must be 64 or 128.
+ *   scale    softmax scale; <= 0 selects 1/sqrt(d).
+ *   out      DEVICE bf16, same layout as q, 16-byte aligned, must not alias
+ *            q, k or v.
+ *   stream   a cudaStream_t (passed as void*), NULL = default stream.
+ * Behaviour: asynchronous on `stream`; returns after the launch.  Argument and
+ * launch errors are returned here.  A device-side wait that runs out (a hung
+ * pipeline) stops that CTA, sets LVSA_DEV_TIMEOUT, and is reported by
+ * lvsa_get_device_status after the stream is synchronised.
+ * Needs an sm_100 (B200-class) device; otherwise LVSA_ERR_UNSUPPORTED.
+ */
+lvsa_status lvsa_attention(const void* q, const void* k, const void* v,
+                           const int32_t* lists, int L, int T, int tokens_per_frame,
+                           int heads, int d, int batch, float scale,
+                           void* out, void* stream);
+
+/*
+ * lvsa_get_device_status -- device status bits (LVSA_DEV_*) of the current
+ * device, OR-ed over every kernel since the last clear.  Synchronises the
+ * device.  clear != 0 resets them to 0 afterwards.
+ */
+lvsa_status lvsa_get_device_status(unsigned int* flags, int clear);
+
+/*
+ * lvsa_set_wait_budget_ns -- time budget of every device-side wait of later
+ * launches (default 4e9 ns).  Values below 1000 ns are raised to 1000 ns.
+ */
+lvsa_status lvsa_set_wait_budget_ns(unsigned long long ns);
+
+/*
+ * lvsa_watchdog_selftest -- launches one CTA that waits on a barrier nobody
+ * arrives on, with the given budget, through the same bounded-wait code the
+ * attention kernel uses.  The wait runs out, sets LVSA_DEV_TIMEOUT and the
+ * kernel returns normally (no trap, no fault).  Used to test failure detection.
+ */
+lvsa_status lvsa_watchdog_selftest(unsigned long long budget_ns, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* lvsa_status_string(int status);
+
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int lvsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LVSA_H */

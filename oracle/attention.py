@@ -26,11 +26,21 @@ import numpy as np
 
 def _f64(x) -> np.ndarray:
     if hasattr(x, "detach"):  # torch tensor -> numpy (CPU), any float dtype
-        x = x.detach().to("cpu")
         import torch
 
-        x = x.to(torch.float64).numpy()
+        x = x.detach().to("cpu").to(torch.float64).numpy()
     return np.asarray(x, dtype=np.float64)
+
+
+def _take(x, b: int, tokens: np.ndarray, h: int) -> np.ndarray:
+    """x[b, tokens, h, :] as float64 (gathered before widening, so a large
+    bf16 torch tensor is never converted whole)."""
+    if hasattr(x, "detach"):
+        import torch
+
+        idx = torch.as_tensor(tokens, dtype=torch.long, device=x.device)
+        return x[b].index_select(0, idx)[:, h, :].detach().to("cpu").to(torch.float64).numpy()
+    return np.asarray(x[b, tokens, h, :], dtype=np.float64)
 
 
 def default_scale(d: int) -> float:
@@ -48,12 +58,10 @@ def sparse_attention_rows(q, k, v, lists, P: int, rows, scale: float | None = No
     """O for the query tokens ``rows`` (iterable of token indices) of every
     batch and head.
 
+    ``q, k, v``: numpy arrays or torch tensors [batch, T*P, heads, d].
     ``lists[t]`` is the frame set A(t) of query frame t.  Returns float64
     [batch, len(rows), heads, d].
     """
-    q = _f64(q)
-    k = _f64(k)
-    v = _f64(v)
     B, Ltok, H, d = q.shape
     sigma = default_scale(d) if scale is None or scale <= 0 else float(scale)
     rows = np.asarray(list(rows), dtype=np.int64)
@@ -64,9 +72,9 @@ def sparse_attention_rows(q, k, v, lists, P: int, rows, scale: float | None = No
         toks = frame_tokens(lists[int(t)], P)
         for b in range(B):
             for h in range(H):
-                Q = q[b, rows[sel], h, :]          # [r, d]
-                K = k[b, toks, h, :]               # [n, d]
-                V = v[b, toks, h, :]               # [n, d]
+                Q = _take(q, b, rows[sel], h)      # [r, d]
+                K = _take(k, b, toks, h)           # [n, d]
+                V = _take(v, b, toks, h)           # [n, d]
                 S = sigma * (Q @ K.T)              # [r, n]
                 m = S.max(axis=1, keepdims=True)
                 E = np.exp(S - m)

@@ -22,12 +22,22 @@ def cuda_available() -> bool:
         return False
 
 
+def load_build_module():
+    """The package's build step, loaded by path (importing the package itself
+    needs the built library)."""
+    import importlib.util
+
+    path = os.path.join(ROOT, "block_sparse_attention_frame_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_lvsa_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 @pytest.fixture(scope="session")
 def lib():
     """The C-ABI library, built in-tree if it is missing or stale."""
-    from block_sparse_attention_frame_b200 import build as libbuild
-
-    libbuild.build_library(quiet=True)
+    load_build_module().build_library(quiet=True)
     import block_sparse_attention_frame_b200 as lvsa
 
     return lvsa
@@ -37,4 +47,6 @@ def lib():
 def gpu_lib(lib):
     if not cuda_available():
         pytest.fail("GPU test collected on a machine without CUDA")
+    # a stuck pipeline gives up after 0.5 s per wait instead of 4 s
+    lib.lvsa_set_wait_budget_ns(500_000_000)
     return lib

@@ -1,0 +1,72 @@
+"""The C-ABI library loads and exports every symbol include/lvsa.h declares;
+argument validation happens before any CUDA call (no GPU needed)."""
+
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "lvsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lvsa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("lvsa_build_frame_lists", "lvsa_attention", "lvsa_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib._lib, name)
+    assert set(lib.EXPORTED) == set(declared_functions())
+
+
+def test_status_strings(lib):
+    assert lib.status_string(0) == "LVSA_OK"
+    assert lib.status_string(4) == "LVSA_ERR_TIMEOUT"
+    assert lib.status_string(99) == "LVSA_ERR_UNKNOWN"
+    assert lib.lvsa_version() >= 100
+
+
+def test_attention_argument_validation_without_gpu(lib):
+    A = 1 << 20  # a 16-byte aligned fake address; validation fails before it is used
+    good = dict(q=A, k=A + 4096, v=A + 8192, lists=A + 12288, L=4, T=8, P=64, H=2, d=64, B=1, scale=0.0,
+                out=A + 16384, stream=0)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return lib.lvsa_attention_raw(a["q"], a["k"], a["v"], a["lists"], a["L"], a["T"], a["P"], a["H"],
+                                      a["d"], a["B"], a["scale"], a["out"], a["stream"])
+
+    INV = lib.LVSA_ERR_INVALID_ARG
+    assert call(q=0) == INV
+    assert call(lists=0) == INV
+    assert call(out=0) == INV
+    assert call(L=0) == INV
+    assert call(L=9) == INV
+    assert call(T=0) == INV
+    assert call(P=0) == INV
+    assert call(H=0) == INV
+    assert call(B=0) == INV
+    assert call(out=A) == INV            # aliases q
+    assert call(q=A + 8) == INV          # not 16-byte aligned
+    assert call(lists=A + 12290) == INV  # int32 misaligned
+    assert call(scale=float("nan")) == INV
+    assert call(T=1 << 20, P=1 << 12) == INV  # T*P overflows int32
+    assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
+    # valid arguments on a machine without a B200: a clean error, never a crash
+    from conftest import cuda_available
+
+    if not cuda_available():
+        assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)

@@ -1,0 +1,189 @@
+"""GPU parity: the CUDA path (C-ABI list builder + sm_100a kernel, called through
+the C ABI) against the fp64 oracle, element by element.
+
+Tolerance (stated for unit-variance bf16 inputs with fp32 accumulation):
+max-abs error <= 2e-2 and mean-abs error <= 2e-3 against the oracle run in
+float64 on the same bf16-rounded inputs.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as OA
+from oracle import lists as OL
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+MEAN_ABS = 2e-3
+
+
+def run_kernel(lib, q, k, v, lists_np, P, scale=0.0):
+    lists = torch.from_numpy(np.ascontiguousarray(lists_np, dtype=np.int32)).cuda()
+    out = lib.lvsa_attention(q, k, v, lists, P, scale=scale)
+    torch.cuda.synchronize()
+    return out
+
+
+def errors(got, ref):
+    err = np.abs(got.astype(np.float64) - ref)
+    return float(err.max()), float(err.mean())
+
+
+def assert_close(got, ref, what=""):
+    mx, mean = errors(got, ref)
+    assert np.isfinite(got).all(), what
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max-abs {mx:.3e} mean-abs {mean:.3e}"
+    return mx, mean
+
+
+def make(T, P, H, d, B=1, seed=0, correlated=True):
+    from block_sparse_attention_frame_b200 import synthetic
+
+    return synthetic.make_custom(T, P, H, d, B=B, seed=seed, device="cuda", frame_correlated_k=correlated)
+
+
+def full_out(out):
+    return out.float().cpu().numpy()
+
+
+def test_tiny_workload_all_steps(gpu_lib):
+    from block_sparse_attention_frame_b200 import synthetic
+
+    w = synthetic.WORKLOADS["tiny"]
+    q32, k32, v32 = synthetic.make_qkv(w, device="cpu", dtype=torch.float32)
+    q, k, v = (x.to(torch.bfloat16) for x in (q32, k32, v32))
+    qd, kd, vd = (x.cuda() for x in (q, k, v))
+    for s in range(w.steps):
+        lists = gpu_lib.lvsa_build_frame_lists(w.T, w.C, w.W, s)
+        out = full_out(run_kernel(gpu_lib, qd, kd, vd, lists, w.P))
+        ref = OA.sparse_attention(q, k, v, OL.frame_lists(w.T, w.C, w.W, s), w.P)
+        assert_close(out, ref, f"tiny step {s}")
+        # also within tolerance of the unrounded fp32 draws
+        ref32 = OA.sparse_attention(q32, k32, v32, OL.frame_lists(w.T, w.C, w.W, s), w.P)
+        assert errors(out, ref32)[0] <= 5e-2
+
+
+def test_negative_control_wrong_step_fails(gpu_lib):
+    from block_sparse_attention_frame_b200 import synthetic
+
+    w = synthetic.WORKLOADS["tiny"]
+    q, k, v = synthetic.make_qkv(w, device="cpu")
+    out = full_out(run_kernel(gpu_lib, q.cuda(), k.cuda(), v.cuda(), gpu_lib.lvsa_build_frame_lists(8, 4, 2, 0),
+                              w.P))
+    ref_wrong = OA.sparse_attention(q, k, v, OL.frame_lists(8, 4, 2, 1), w.P)
+    mx, mean = errors(out, ref_wrong)
+    assert mx > MAX_ABS and mean > MEAN_ABS
+
+
+@pytest.mark.parametrize("T,P,H,d,B,C,W,s", [
+    (6, 200, 3, 128, 2, 3, 1, 4),     # 2 query tiles per frame (128 + 72 rows), ragged K/V runs
+    (7, 300, 2, 64, 1, 4, 2, 3),      # d = 64, 3 query tiles (128+128+44)
+    (10, 129, 2, 128, 1, 5, 2, 7),    # one-row tail tiles everywhere
+    (5, 17, 4, 128, 1, 2, 1, 1),      # tokens per frame below one tile
+    (9, 256, 1, 128, 1, 9, 3, 0),     # C = T: dense
+    (12, 96, 2, 128, 1, 5, 5, 2),     # G = 0: pure sliding window
+    (1, 1000, 2, 128, 1, 21, 9, 0),   # T = 1
+])
+def test_ragged_shapes_full_parity(gpu_lib, T, P, H, d, B, C, W, s):
+    q, k, v = make(T, P, H, d, B=B, seed=T * 1000 + P)
+    lists = gpu_lib.lvsa_build_frame_lists(T, C, W, s)
+    out = full_out(run_kernel(gpu_lib, q, k, v, lists, P))
+    ref = OA.sparse_attention(q, k, v, OL.frame_lists(T, C, W, s), P)
+    assert_close(out, ref, f"T={T} P={P} d={d}")
+
+
+def test_dense_lists_equal_full_attention(gpu_lib):
+    T, P, H, d = 4, 160, 2, 128
+    q, k, v = make(T, P, H, d, seed=77)
+    out = full_out(run_kernel(gpu_lib, q, k, v, gpu_lib.lvsa_build_frame_lists(T, T, 1, 0), P))
+    assert_close(out, OA.dense_attention(q, k, v), "dense")
+
+
+def test_explicit_scale(gpu_lib):
+    T, P, H, d = 5, 130, 2, 64
+    q, k, v = make(T, P, H, d, seed=5)
+    lists = gpu_lib.lvsa_build_frame_lists(T, 3, 1, 2)
+    out = full_out(run_kernel(gpu_lib, q, k, v, lists, P, scale=0.05))
+    assert_close(out, OA.sparse_attention(q, k, v, OL.frame_lists(T, 3, 1, 2), P, scale=0.05), "scale")
+
+
+def test_large_logits_rescale_path(gpu_lib):
+    # keys growing along the list order force many running-max updates (O rescales)
+    T, P, H, d = 6, 256, 1, 128
+    q, k, v = make(T, P, H, d, seed=8)
+    ramp = torch.linspace(0, 6, T * P, device="cuda").view(1, T * P, 1, 1)
+    k = (k.float() + ramp * q.float().mean(dim=1, keepdim=True)).to(torch.bfloat16).contiguous()
+    q = (q.float() * 2).to(torch.bfloat16).contiguous()
+    lists = gpu_lib.lvsa_build_frame_lists(T, 4, 2, 3)
+    out = full_out(run_kernel(gpu_lib, q, k, v, lists, P))
+    assert_close(out, OA.sparse_attention(q, k, v, OL.frame_lists(T, 4, 2, 3), P), "rescale")
+
+
+def test_unsorted_lists_same_result(gpu_lib):
+    T, P, H, d = 8, 150, 2, 128
+    q, k, v = make(T, P, H, d, seed=3)
+    lists = gpu_lib.lvsa_build_frame_lists(T, 4, 2, 5)
+    rev = np.ascontiguousarray(lists[:, ::-1])
+    a = full_out(run_kernel(gpu_lib, q, k, v, lists, P))
+    b = full_out(run_kernel(gpu_lib, q, k, v, rev, P))
+    assert_close(b, a.astype(np.float64), "list order")
+
+
+def test_bad_list_entry_flagged_and_skipped(gpu_lib):
+    T, P, H, d = 6, 64, 1, 64
+    q, k, v = make(T, P, H, d, seed=4)
+    gpu_lib.lvsa_get_device_status(clear=True)
+    lists = gpu_lib.lvsa_build_frame_lists(T, 3, 1, 0).copy()
+    good = [list(r) for r in lists]
+    lists[2, 1] = 99  # out of range: skipped, status bit set
+    good[2] = [f for j, f in enumerate(good[2]) if j != 1]
+    out = full_out(run_kernel(gpu_lib, q, k, v, lists, P))
+    assert gpu_lib.lvsa_get_device_status(clear=True) & gpu_lib.LVSA_DEV_BAD_LIST
+    assert_close(out, OA.sparse_attention(q, k, v, good, P), "bad list")
+
+
+def test_watchdog_times_out_and_context_survives(gpu_lib):
+    gpu_lib.lvsa_get_device_status(clear=True)
+    gpu_lib.lvsa_watchdog_selftest(2_000_000)  # 2 ms budget on a barrier nobody arrives on
+    torch.cuda.synchronize()
+    assert gpu_lib.lvsa_get_device_status(clear=True) & gpu_lib.LVSA_DEV_TIMEOUT
+    # the context is still usable
+    test_dense_lists_equal_full_attention(gpu_lib)
+    assert gpu_lib.lvsa_get_device_status(clear=True) == 0
+
+
+def sample_rows(T, P, seed, per_frame=40):
+    g = np.random.default_rng(seed)
+    frames = sorted(set([0, 1, T // 2, T - 2, T - 1] + list(g.choice(T, 3, replace=False))))
+    base = sorted(set([0, 1, 127, 128, P - 25, P - 24, P - 1] + list(range(min(1535, P - 1), P, 8))))
+    rows = []
+    for f in frames:
+        extra = g.choice(P, max(0, per_frame - len(base)), replace=False)
+        rows += [f * P + r for r in sorted(set(base) | set(int(x) for x in extra))]
+    return rows
+
+
+@pytest.mark.parametrize("name,steps", [
+    ("wan1.3b_1x", [0]),
+    ("wan1.3b_6x", [0, 17, 49]),
+    ("hunyuan1.5_1.5x", [0, 2, 31]),
+    ("wan14b_6x", [5]),
+])
+def test_full_size_workloads_sampled_rows(gpu_lib, name, steps):
+    from block_sparse_attention_frame_b200 import synthetic
+
+    w = synthetic.WORKLOADS[name]
+    q, k, v = synthetic.make_qkv(w, device="cuda")
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    rows = sample_rows(w.T, w.P, seed=w.seed)
+    for s in steps:
+        lists = gpu_lib.lvsa_build_frame_lists(w.T, w.C, w.W, s)
+        out = run_kernel(gpu_lib, q, k, v, lists, w.P)
+        got = out[:, rows].float().cpu().numpy()
+        ref = OA.sparse_attention_rows(qc, kc, vc, OL.frame_lists(w.T, w.C, w.W, s), w.P, rows)
+        assert_close(got, ref, f"{name} step {s}")
+        assert torch.isfinite(out).all()
+        del out
+    torch.cuda.empty_cache()
