@@ -295,6 +295,11 @@ def run_lvsa(args, rank, world, local):
         raise RuntimeError(f"device status {status:#x} after the timed region")
     ms_per_step = elapsed_ms / args.steps
     value = world * F * args.steps / (elapsed_ms * 1e-3) / 1e12
+    if args.kernel_only:
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "value": value, "unit": "TFLOP/s", "ms_per_step": ms_per_step,
+                              "kernel_ms": kernel_ms, "clocks": clocks.summary()}), flush=True)
+        return 0
 
     # ---------------------------------------------------------------- dense control (same kernel, C = T)
     dense_lists = torch.from_numpy(lvsa.lvsa_build_frame_lists(w.T, w.T, 1, 0)).to(dev)
@@ -407,6 +412,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="lvsa", choices=["lvsa", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time the device path only and print a short line (for profiling runs)")
     ap.add_argument("--ref-seconds", type=float, default=0.0, help="reference arm: CPU seconds per step")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps; the JSON reports the count used
