@@ -35,7 +35,8 @@ LVSA_DEV_BAD_LIST = 0x2
 
 EXPORTED = [
     "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_get_device_status",
-    "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_status_string", "lvsa_version",
+    "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_exp2_fma_eval", "lvsa_status_string",
+    "lvsa_version",
 ]
 
 
@@ -47,7 +48,7 @@ class LvsaError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m block_sparse_attention_frame_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python block_sparse_attention_frame_b200/build.py` "
         "(there is no fallback path)")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -68,6 +69,8 @@ _lib.lvsa_set_wait_budget_ns.argtypes = [_c_ull]
 _lib.lvsa_set_wait_budget_ns.restype = _c_int
 _lib.lvsa_watchdog_selftest.argtypes = [_c_ull, _c_vp]
 _lib.lvsa_watchdog_selftest.restype = _c_int
+_lib.lvsa_exp2_fma_eval.argtypes = [_c_vp, _c_vp, _c_int, _c_vp]
+_lib.lvsa_exp2_fma_eval.restype = _c_int
 _lib.lvsa_status_string.argtypes = [_c_int]
 _lib.lvsa_status_string.restype = ctypes.c_char_p
 _lib.lvsa_version.argtypes = []
@@ -181,3 +184,16 @@ def lvsa_watchdog_selftest(budget_ns: int, stream=None) -> None:
 
     _check("lvsa_watchdog_selftest",
            _lib.lvsa_watchdog_selftest(int(budget_ns), _stream_ptr(stream, torch.cuda.current_device())))
+
+
+def lvsa_exp2_fma_eval(x, stream=None):
+    """The kernel's FMA-pipe 2^x on a CUDA float32 tensor (test hook)."""
+    import torch
+
+    if x.device.type != "cuda" or x.dtype != torch.float32 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    with torch.cuda.device(x.device):
+        _check("lvsa_exp2_fma_eval",
+               _lib.lvsa_exp2_fma_eval(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream, x.device)))
+    return y

@@ -1,6 +1,6 @@
 """Build step of the in-tree C-ABI library ``liblvsa.so`` (sm_100a).
 
-``python -m block_sparse_attention_frame_b200.build [--force] [--ptxas-v]``
+``python block_sparse_attention_frame_b200/build.py [--force] [--ptxas-v]``
 compiles ``csrc/*.cpp`` and ``csrc/*.cu`` with nvcc for sm_100a into
 ``block_sparse_attention_frame_b200/liblvsa.so``.  nvcc cross-compiles, so this
 runs on a machine without a GPU.

@@ -41,15 +41,19 @@ using namespace sm100;
 
 constexpr int kBM = 128;          // query rows per tile = MMA M
 constexpr int kBN = 128;          // keys per K/V tile = largest MMA N of QK^T
-constexpr int kThreads = 192;     // 4 softmax warps + TMA warp + MMA warp
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
-constexpr int kTmemCols = 512;
-constexpr int kSCol0 = 0;         // S/P buffer 0: TMEM columns [0,128)
-constexpr int kSCol1 = 128;       // S/P buffer 1: TMEM columns [128,256)
-constexpr int kOCol = 256;        // O accumulator: TMEM columns [256, 256+d)
+constexpr int kQTiles = 2;        // query tiles per CTA, sharing every K/V tile
+constexpr int kThreads = 384;     // warps 0-3: softmax tile 0, 4-7: softmax tile 1, 8: TMA, 9: MMA, 10-11 idle
+// Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup drops to 72 and the
+// two softmax warpgroups rise to 216: 2 x 128 x 216 + 128 x 72 = 64512.
+constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsControl = 72;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kTmemCols = 512;    // S/P of tile i: columns [128 i, 128 i + 128); O of tile i: [256 + 128 i, ...)
+constexpr int kOCol0 = 256;
 constexpr int kChunkBytes = kBM * 128;    // one 128-byte-wide swizzle column of a 128-row tile
 constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the max grows by > 2^8
+constexpr int kPolyEvery = 4;             // every 4th element pair takes the FMA-pipe exp2
 
 template <int D>
 struct Cfg {
@@ -57,11 +61,12 @@ struct Cfg {
   static constexpr int kTileBytes = kBM * D * 2;
   static constexpr int kSlots = (D == 128) ? 5 : 10;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffRing = kTileBytes;
+  static constexpr int kOffRing = kQTiles * kTileBytes;
   static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
   static constexpr int kBarBytes = 512;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(8 * (1 + 2 * kSlots + 7) + 8 <= kBarBytes, "barrier area");
 };
 
 struct KernelParams {
@@ -71,7 +76,7 @@ struct KernelParams {
   __nv_bfloat16* out;
   const int32_t* lists;
   int T, P, H, L;
-  int qtiles;        // ceil(P / 128)
+  int qblocks;       // ceil(P / 256): CTAs per query frame
   float scale_log2;  // softmax scale * log2(e)
   unsigned long long wait_ns;
 };
@@ -146,6 +151,93 @@ struct TileWalk {
   }
 };
 
+// ------------------------------------------------------------------ softmax of one S tile
+// Thread = one query row.  Loads the row of S from TMEM, masks columns past the
+// run end, updates the running max lazily (rescaling the row of O in TMEM when
+// needed), writes P = 2^(scale*log2e*s - m) as bf16 over the S columns and
+// returns the row sum of P through `l`.
+template <int D>
+__device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int nv, int j, float sl2, float& m,
+                                             float& l, uint64_t* bar_o, const Watch& w) {
+  float s[kBN];
+  tmem_ld32(s_tmem + 0, s + 0);
+  if (nv > 32) tmem_ld32(s_tmem + 32, s + 32);
+  if (nv > 64) tmem_ld32(s_tmem + 64, s + 64);
+  if (nv > 96) tmem_ld32(s_tmem + 96, s + 96);
+  tmem_wait_ld_regs(s + 0);
+  tmem_wait_ld_regs(s + 32);
+  tmem_wait_ld_regs(s + 64);
+  tmem_wait_ld_regs(s + 96);
+  const bool partial = nv < kBN;
+  if (partial) {
+#pragma unroll
+    for (int i = 0; i < kBN; ++i)
+      if (i >= nv) s[i] = -INFINITY;
+  }
+  // row max: 8 chains of 3-input max
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = s[k];
+#pragma unroll
+  for (int i = 8; i < 120; i += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 8 + k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[120 + k]);
+  const float tile_max = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7])) * sl2;
+
+  float alpha = 1.f;
+  if (tile_max > m + kRescaleLog2) {
+    alpha = ex2(m - tile_max);
+    l *= alpha;
+    m = tile_max;
+  }
+  if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+    // O holds PV(0..j-1): wait for PV(j-1), then rescale this thread's row
+    if (!__all_sync(0xffffffffu, wait_bounded(bar_o, (j - 1) & 1, w))) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      tmem_ld32(o_tmem + 32 * c, o);
+      tmem_wait_ld_regs(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] *= alpha;
+      tmem_st32(o_tmem + 32 * c, o);
+    }
+  }
+
+  const float2 scale2 = make_float2(sl2, sl2);
+  const float2 negm2 = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c == 0 || nv > 32 * c) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 x = ffma2(make_float2(s[32 * c + 2 * i], s[32 * c + 2 * i + 1]), scale2, negm2);
+        float2 e;
+        if (!partial && (i % kPolyEvery) == kPolyEvery - 1) {
+          e = exp2_fma2(x);
+        } else {
+          e.x = ex2(x.x);
+          e.y = ex2(x.y);
+        }
+        acc[i & 3] = fadd2(acc[i & 3], e);
+        pk[i] = pack_bf16x2(e.x, e.y);
+      }
+      tmem_st16(s_tmem + 16 * c, pk);  // P overwrites the first half of the S columns
+    }
+  }
+  const float2 t01 = fadd2(acc[0], acc[1]);
+  const float2 t23 = fadd2(acc[2], acc[3]);
+  const float2 tt = fadd2(t01, t23);
+  l += tt.x + tt.y;
+  return true;
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __grid_constant__ KernelParams p) {
@@ -158,19 +250,21 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   uint64_t* bar_q = bars;
   uint64_t* bar_full = bars + 1;
   uint64_t* bar_empty = bar_full + Cf::kSlots;
-  uint64_t* bar_s = bar_empty + Cf::kSlots;  // [2] S(j) ready in TMEM
-  uint64_t* bar_p = bar_s + 2;               // [2] P(j) written to TMEM (128 arrivals)
-  uint64_t* bar_o = bar_p + 2;               // PV(j) finished
-  uint64_t* bar_drain = bar_o + 1;           // all MMAs of the CTA finished
+  uint64_t* bar_s = bar_empty + Cf::kSlots;  // [2] S_i(j) ready in TMEM
+  uint64_t* bar_p = bar_s + 2;               // [2] P_i(j) written to TMEM (128 arrivals)
+  uint64_t* bar_o = bar_p + 2;               // [2] PV_i(j) finished
+  uint64_t* bar_drain = bar_o + 2;           // all MMAs of the CTA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % p.qtiles;
-  const int t = blockIdx.x / p.qtiles;
+  const int qb = blockIdx.x % p.qblocks;
+  const int t = blockIdx.x / p.qblocks;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
+  const int row0 = qb * kQTiles * kBM;        // first query row (within frame t) of this CTA
+  const bool has1 = row0 + kBM < p.P;         // the second query tile has rows
   const int32_t* list = p.lists + static_cast<size_t>(t) * p.L;
 
   if (threadIdx.x == 0) {
@@ -179,11 +273,11 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       mbar_init(bar_full + i, 1);
       mbar_init(bar_empty + i, 1);
     }
-    mbar_init(bar_s + 0, 1);
-    mbar_init(bar_s + 1, 1);
-    mbar_init(bar_p + 0, 4 * 32);
-    mbar_init(bar_p + 1, 4 * 32);
-    mbar_init(bar_o, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_s + i, 1);
+      mbar_init(bar_p + i, 4 * 32);
+      mbar_init(bar_o + i, 1);
+    }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -203,15 +297,21 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   const uint32_t tmem = *tmem_slot;
   const Watch w{p.wait_ns, abort_flag};
 
+  if (warp >= 8) {
+  regs_dec<kRegsControl>();
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int col0 = h * D;
-      const int qrow = t * p.P + qt * kBM;
-      mbar_arrive_expect_tx(bar_q, Cf::kTileBytes);
+      const int qrow = t * p.P + row0;
+      mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * Cf::kTileBytes);
 #pragma unroll
       for (int c = 0; c < Cf::kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &p.tm_q, bar_q, col0 + c * 64, qrow, b);
-
+      if (has1) {
+#pragma unroll
+        for (int c = 0; c < Cf::kChunks; ++c)
+          tma_load_3d(sQ + Cf::kTileBytes + c * kChunkBytes, &p.tm_q, bar_q, col0 + c * 64, qrow + kBM, b);
+      }
       int issued = 0;
       bool ok = true;
       auto load = [&](const CUtensorMap* tm, int tok) {
@@ -227,15 +327,13 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         for (int c = 0; c < Cf::kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, tm, bar_full + slot, col0 + c * 64, tok, b);
         ++issued;
       };
-      // consumption order of the MMA warp: K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1)
+      // consumption order of the MMA warp: K0, V0, K1, V1, ...
       TileWalk walk(list, p.L, p.T, p.P);
-      int tok, nv, prev = -1;
+      int tok, nv;
       while (ok && walk.next(tok, nv)) {
         load(&p.tm_k, tok);
-        if (ok && prev >= 0) load(&p.tm_v, prev);
-        prev = tok;
+        if (ok) load(&p.tm_v, tok);
       }
-      if (ok && prev >= 0) load(&p.tm_v, prev);
       if (walk.bad) atomicOr(&g_lvsa_dev_status, LVSA_DEV_BAD_LIST);
       if (!ok) {
         // stopped early: let every copy still in flight land before the CTA exits
@@ -246,169 +344,153 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
+    // Per K/V tile j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while softmax 1 works on S_1(j)
+    // the tensor core runs tile 0's products, and the other way round.
     if (lane == 0) {
       const uint32_t sq = smem_u32(sQ);
       const uint32_t sr = smem_u32(sRing);
       const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
-      int consumed = 0;
-      bool ok = wait_bounded(bar_q, 0, w);
-      auto issue_pv = [&](int i, int n_mma) {
-        const int slot = consumed % Cf::kSlots;
-        const uint32_t phase = (consumed / Cf::kSlots) & 1;
-        if (!wait_bounded(bar_p + (i & 1), (i >> 1) & 1, w) || !wait_bounded(bar_full + slot, phase, w)) {
-          ok = false;
-          return;
-        }
-        tc_fence_after();
-        const uint32_t v_addr = sr + slot * Cf::kTileBytes;
-        const uint32_t p_tmem = tmem + ((i & 1) ? kSCol1 : kSCol0);
-        for (int kk = 0; kk < n_mma / 16; ++kk) {
-          // B = V tile, MN-major (d contiguous): 64-wide d chunks 16 KB apart (LBO), 8-key groups 1 KB apart (SBO)
-          const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, kChunkBytes, 1024);
-          mma_ts(tmem + kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(bar_empty + slot);
-        mma_commit(bar_o);
-        ++consumed;
-      };
-      TileWalk walk(list, p.L, p.T, p.P);
-      int tok, nv, j = 0, prev_n = 0;
-      while (ok && walk.next(tok, nv)) {
-        const int n_mma = (nv + 15) & ~15;
-        const int slot = consumed % Cf::kSlots;
-        const uint32_t phase = (consumed / Cf::kSlots) & 1;
-        if (!wait_bounded(bar_full + slot, phase, w)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_addr = sr + slot * Cf::kTileBytes;
-        const uint32_t idesc_qk = idesc_bf16_f32(kBM, n_mma, false);
-        const uint32_t s_tmem = tmem + ((j & 1) ? kSCol1 : kSCol0);
+      auto qk = [&](int i, uint32_t k_addr, int n_mma) {
+        const uint32_t q_addr = sq + i * Cf::kTileBytes;
+        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma, false);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // A = Q, B = K, both K-major: 16-element (32-byte) steps inside a 128-byte swizzle row
           const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          mma_ss(s_tmem, smem_desc_sw128(sq + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(tmem + 128 * i, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
+                 idesc, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar_empty + slot);
-        mma_commit(bar_s + (j & 1));
-        ++consumed;
-        if (j > 0) issue_pv(j - 1, prev_n);
-        prev_n = n_mma;
-        ++j;
+      };
+      auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate) {
+        for (int kk = 0; kk < n_mma / 16; ++kk) {
+          // B = V tile, MN-major (d contiguous): 64-wide d chunks 16 KB apart (LBO), 8-key groups 1 KB apart (SBO)
+          const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, kChunkBytes, 1024);
+          mma_ts(tmem + kOCol0 + 128 * i, tmem + 128 * i + kk * 8, bdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto slot_of = [&](int idx) { return idx % Cf::kSlots; };
+      auto wait_full = [&](int idx) { return wait_bounded(bar_full + slot_of(idx), (idx / Cf::kSlots) & 1, w); };
+
+      int cidx = 0;
+      bool ok = wait_bounded(bar_q, 0, w);
+      TileWalk walk(list, p.L, p.T, p.P);
+      int tok, nv;
+      if (ok && walk.next(tok, nv)) {
+        int n_cur = (nv + 15) & ~15;
+        const int k0 = cidx++;
+        ok = wait_full(k0);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t k_addr = sr + slot_of(k0) * Cf::kTileBytes;
+          qk(0, k_addr, n_cur);
+          mma_commit(bar_s + 0);
+          if (has1) {
+            qk(1, k_addr, n_cur);
+            mma_commit(bar_s + 1);
+          }
+          mma_commit(bar_empty + slot_of(k0));
+        }
+        for (int j = 0; ok; ++j) {
+          int tok_n, nv_n;
+          const bool has_next = walk.next(tok_n, nv_n);
+          const int n_next = (nv_n + 15) & ~15;
+          const int vi = cidx++;
+          const uint32_t v_addr = sr + slot_of(vi) * Cf::kTileBytes;
+          if (!wait_bounded(bar_p + 0, j & 1, w) || !wait_full(vi)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv(0, v_addr, n_cur, j > 0);
+          mma_commit(bar_o + 0);
+          int ki = -1;
+          uint32_t k_addr = 0;
+          if (has_next) {
+            ki = cidx++;
+            k_addr = sr + slot_of(ki) * Cf::kTileBytes;
+            if (!wait_full(ki)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            qk(0, k_addr, n_next);
+            mma_commit(bar_s + 0);
+          }
+          if (has1) {
+            if (!wait_bounded(bar_p + 1, j & 1, w)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            pv(1, v_addr, n_cur, j > 0);
+            mma_commit(bar_o + 1);
+          }
+          mma_commit(bar_empty + slot_of(vi));
+          if (!has_next) break;
+          if (has1) {
+            qk(1, k_addr, n_next);
+            mma_commit(bar_s + 1);
+          }
+          mma_commit(bar_empty + slot_of(ki));
+          n_cur = n_next;
+        }
       }
-      if (ok && j > 0) issue_pv(j - 1, prev_n);
       // every MMA issued must be complete before TMEM is released
       mma_commit(bar_drain);
       wait_drain(bar_drain, 0, p.wait_ns);
     }
     __syncwarp();
+  }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue (warps 0-3)
-    const int r = threadIdx.x;  // query row of the tile = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t o_tmem = tmem + lane_off + kOCol;
-    const float sl2 = p.scale_log2;
-    float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale by < 8)
-    float l = 0.f;        // running sum of exp2(scaled s - m)
-    bool ok = true;
-    int j = 0;
-    TileWalk walk(list, p.L, p.T, p.P);
-    int tok, nv;
-    while (walk.next(tok, nv)) {
-      const uint32_t s_tmem = tmem + lane_off + ((j & 1) ? kSCol1 : kSCol0);
-      ok = __all_sync(0xffffffffu, wait_bounded(bar_s + (j & 1), (j >> 1) & 1, w));
-      if (!ok) break;
-      tc_fence_after();
-      float s[kBN];
-      tmem_ld32(s_tmem + 0, s + 0);
-      if (nv > 32) tmem_ld32(s_tmem + 32, s + 32);
-      if (nv > 64) tmem_ld32(s_tmem + 64, s + 64);
-      if (nv > 96) tmem_ld32(s_tmem + 96, s + 96);
-      tmem_wait_ld_regs(s + 0);
-      tmem_wait_ld_regs(s + 32);
-      tmem_wait_ld_regs(s + 64);
-      tmem_wait_ld_regs(s + 96);
-      if (nv < kBN) {
-#pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i >= nv) s[i] = -INFINITY;
-      }
-      float mx[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx[u] = s[u];
-#pragma unroll
-      for (int i = 8; i < kBN; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-      const float tile_max = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * sl2;
-      float alpha = 1.f;
-      if (tile_max > m + kRescaleLog2) {
-        alpha = ex2(m - tile_max);
-        l *= alpha;
-        m = tile_max;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O holds PV(0..j-1): wait for PV(j-1), then rescale this thread's row
-        ok = __all_sync(0xffffffffu, wait_bounded(bar_o, (j - 1) & 1, w));
+    regs_inc<kRegsSoftmax>();
+    // ------------------------------------------------------------ softmax + epilogue (warps 0-7)
+    const int qi = warp >> 2;            // query tile of this warpgroup
+    const int r = threadIdx.x & 127;     // row within the tile = TMEM lane
+    if (qi == 0 || has1) {
+      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const uint32_t s_tmem = tmem + lane_off + 128 * qi;
+      const uint32_t o_tmem = tmem + lane_off + kOCol0 + 128 * qi;
+      float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale by < 8)
+      float l = 0.f;        // running sum of 2^(scaled s - m)
+      bool ok = true;
+      int j = 0;
+      TileWalk walk(list, p.L, p.T, p.P);
+      int tok, nv;
+      while (walk.next(tok, nv)) {
+        ok = __all_sync(0xffffffffu, wait_bounded(bar_s + qi, j & 1, w));
         if (!ok) break;
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(o_tmem + 32 * c, o);
-          tmem_wait_ld_regs(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(o_tmem + 32 * c, o);
-        }
+        ok = softmax_tile<D>(s_tmem, o_tmem, nv, j, p.scale_log2, m, l, bar_o + qi, w);
+        if (!ok) break;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p + qi);
+        ++j;
       }
-      const float neg_m = -m;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      if (ok && j > 0) {
+        ok = __all_sync(0xffffffffu, wait_bounded(bar_o + qi, (j - 1) & 1, w));
+        if (ok) {
+          tc_fence_after();
+          const float inv_l = 1.f / l;
+          const int row = row0 + qi * kBM + r;
+          const bool valid = row < p.P;
+          const size_t ltok = static_cast<size_t>(p.T) * p.P;
+          __nv_bfloat16* dst =
+              p.out + ((static_cast<size_t>(b) * ltok + static_cast<size_t>(t) * p.P + row) * p.H + h) * D;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (c == 0 || nv > 32 * c) {
-          uint32_t pk[16];
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(o_tmem + 32 * c, o);
+            tmem_wait_ld_regs(o);
+            if (valid) {
+              uint4 pk[4];
+              uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float e0 = ex2(fmaf(s[32 * c + 2 * i], sl2, neg_m));
-            const float e1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, neg_m));
-            ls[i & 3] += e0 + e1;
-            pk[i] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(s_tmem + 16 * c, pk);  // P overwrites the first half of the S buffer
-        }
-      }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar_p + (j & 1));
-      ++j;
-    }
-    if (ok && j > 0) {
-      ok = __all_sync(0xffffffffu, wait_bounded(bar_o, (j - 1) & 1, w));
-      if (ok) {
-        tc_fence_after();
-        const float inv_l = 1.f / l;
-        const int row = qt * kBM + r;
-        const bool valid = row < p.P;
-        const size_t ltok = static_cast<size_t>(p.T) * p.P;
-        __nv_bfloat16* dst =
-            p.out + ((static_cast<size_t>(b) * ltok + static_cast<size_t>(t) * p.P + row) * p.H + h) * D;
+              for (int i = 0; i < 16; ++i) pw[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+              uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(o_tmem + 32 * c, o);
-          tmem_wait_ld_regs(o);
-          if (valid) {
-            uint4 pk[4];
-            uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pw[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+              for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+            }
           }
         }
       }
@@ -435,6 +517,17 @@ __global__ void watchdog_selftest_kernel(unsigned long long budget_ns) {
   __syncthreads();
   const Watch w{budget_ns, &abort_flag};
   (void)__all_sync(0xffffffffu, wait_bounded(&bar, 0, w));
+}
+
+__global__ void exp2_fma_eval_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (2 * i + 1 < n) {
+    const float2 r = exp2_fma2(make_float2(x[2 * i], x[2 * i + 1]));
+    y[2 * i] = r.x;
+    y[2 * i + 1] = r.y;
+  } else if (2 * i < n) {
+    y[2 * i] = exp2_fma2(make_float2(x[2 * i], 0.f)).x;
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -488,7 +581,7 @@ lvsa_status launch(const KernelParams& kp, int B, cudaStream_t stream, int dev) 
       g_attr_set[di][dev] = true;
     }
   }
-  dim3 grid(static_cast<unsigned>(kp.T * kp.qtiles), static_cast<unsigned>(kp.H), static_cast<unsigned>(B));
+  dim3 grid(static_cast<unsigned>(kp.T * kp.qblocks), static_cast<unsigned>(kp.H), static_cast<unsigned>(B));
   lvsa_attention_kernel<D><<<grid, kThreads, Cf::kSmemBytes, stream>>>(kp);
   return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
 }
@@ -513,8 +606,8 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lists) & 3u))
     return LVSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return LVSA_ERR_UNSUPPORTED;
-  const int qtiles = (P + kBM - 1) / kBM;
-  if (static_cast<long long>(T) * qtiles > INT_MAX) return LVSA_ERR_INVALID_ARG;
+  const int qblocks = (P + kQTiles * kBM - 1) / (kQTiles * kBM);
+  if (static_cast<long long>(T) * qblocks > INT_MAX) return LVSA_ERR_INVALID_ARG;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LVSA_ERR_CUDA;
@@ -533,7 +626,7 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   kp.P = P;
   kp.H = heads;
   kp.L = L;
-  kp.qtiles = qtiles;
+  kp.qblocks = qblocks;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   kp.scale_log2 = sc * 1.4426950408889634f;
   kp.wait_ns = g_wait_ns;
@@ -563,6 +656,15 @@ extern "C" lvsa_status lvsa_watchdog_selftest(unsigned long long budget_ns, void
   if (budget_ns < 1000ull) budget_ns = 1000ull;
   if (budget_ns > 10000000000ull) return LVSA_ERR_INVALID_ARG;
   lvsa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_ns);
+  return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
+}
+
+extern "C" lvsa_status lvsa_exp2_fma_eval(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n < 0 || (reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u))
+    return LVSA_ERR_INVALID_ARG;
+  if (n == 0) return LVSA_OK;
+  const int pairs = (n + 1) / 2;
+  lvsa::exp2_fma_eval_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
 }
 

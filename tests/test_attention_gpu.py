@@ -187,3 +187,15 @@ def test_full_size_workloads_sampled_rows(gpu_lib, name, steps):
         assert torch.isfinite(out).all()
         del out
     torch.cuda.empty_cache()
+
+
+def test_fma_pipe_exp2_against_cuda_exp2(gpu_lib):
+    # the kernel's polynomial 2^x versus CUDA's exp2 over the whole range it is used on
+    x = torch.cat([torch.linspace(-125.0, 9.0, 2_000_001, device="cuda"),
+                   torch.linspace(-1.0, 1.0, 100_001, device="cuda"),
+                   torch.tensor([-125.0, -0.5, 0.0, 0.5, 8.0, -300.0, float("-inf")], device="cuda")])
+    y = gpu_lib.lvsa_exp2_fma_eval(x.contiguous())
+    ref = torch.exp2(x.double().clamp(min=-125.0))
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel <= 1e-4, rel
+    assert (y > 0).all() and torch.isfinite(y).all()
