@@ -43,17 +43,17 @@ constexpr int kBM = 128;          // query rows per tile = MMA M
 constexpr int kBN = 128;          // keys per K/V tile = largest MMA N of QK^T
 constexpr int kQTiles = 2;        // query tiles per CTA, sharing every K/V tile
 constexpr int kThreads = 384;     // warps 0-3: softmax tile 0, 4-7: softmax tile 1, 8: TMA, 9: MMA, 10-11 idle
-// Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup drops to 72 and the
-// two softmax warpgroups rise to 216: 2 x 128 x 216 + 128 x 72 = 64512.
-constexpr uint32_t kRegsSoftmax = 216;
-constexpr uint32_t kRegsControl = 72;
+// Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup drops to 88 and the
+// two softmax warpgroups rise to 208: 2 x 128 x 208 + 128 x 88 = 64512.
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsControl = 88;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kTmemCols = 512;    // S/P of tile i: columns [128 i, 128 i + 128); O of tile i: [256 + 128 i, ...)
 constexpr int kOCol0 = 256;
 constexpr int kChunkBytes = kBM * 128;    // one 128-byte-wide swizzle column of a 128-row tile
 constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the max grows by > 2^8
-constexpr int kPolyEvery = 4;             // every 4th element pair takes the FMA-pipe exp2
+constexpr int kPolyEvery = 0;             // every kPolyEvery-th element pair takes the FMA-pipe exp2 (0: none)
 
 template <int D>
 struct Cfg {
@@ -78,12 +78,18 @@ struct KernelParams {
   int T, P, H, L;
   int qblocks;       // ceil(P / 256): CTAs per query frame
   float scale_log2;  // softmax scale * log2(e)
-  unsigned long long wait_ns;
+  long long wait_cycles;
 };
 
 // ------------------------------------------------------------------ bounded waits
+// The budget is counted in SM clock cycles (a ns budget converted at 2 GHz, so at
+// lower clocks it lasts longer in wall time).  The cycle counter and the abort
+// flag are only looked at every 64 polls: the poll itself must stay cheap, since
+// a slow poll delays the hand-off it waits for.
+constexpr double kBudgetCyclesPerNs = 2.0;
+
 struct Watch {
-  unsigned long long budget_ns;
+  long long budget_cycles;
   volatile int* abort_flag;  // shared memory, CTA-wide
 };
 
@@ -91,23 +97,25 @@ struct Watch {
 // CTA already gave up.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Watch& w) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*w.abort_flag) return false;
-    if (global_timer_ns() - t0 > w.budget_ns) {
-      *w.abort_flag = 1;
-      atomicOr(&g_lvsa_dev_status, LVSA_DEV_TIMEOUT);
-      return false;
+    if ((it & 63u) == 0) {
+      if (*w.abort_flag) return false;
+      if (clock64() - t0 > w.budget_cycles) {
+        *w.abort_flag = 1;
+        atomicOr(&g_lvsa_dev_status, LVSA_DEV_TIMEOUT);
+        return false;
+      }
     }
   }
 }
 
 // Used only while shutting down after an abort: ignores the abort flag.
-__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, unsigned long long budget_ns) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > budget_ns) {
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long long budget_cycles) {
+  const long long t0 = clock64();
+  for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it) {
+    if ((it & 63u) == 63u && clock64() - t0 > budget_cycles) {
       atomicOr(&g_lvsa_dev_status, LVSA_DEV_TIMEOUT);
       return;
     }
@@ -219,7 +227,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       for (int i = 0; i < 16; ++i) {
         const float2 x = ffma2(make_float2(s[32 * c + 2 * i], s[32 * c + 2 * i + 1]), scale2, negm2);
         float2 e;
-        if (!partial && (i % kPolyEvery) == kPolyEvery - 1) {
+        if (kPolyEvery > 0 && !partial && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
           e = exp2_fma2(x);
         } else {
           e.x = ex2(x.x);
@@ -295,15 +303,17 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const Watch w{p.wait_ns, abort_flag};
+  const Watch w{p.wait_cycles, abort_flag};
 
   if (warp >= 8) {
   regs_dec<kRegsControl>();
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const int col0 = h * D;
-      const int qrow = t * p.P + row0;
+    // The whole warp walks the list (warp-uniform control flow); one elected
+    // lane arms the barriers and issues the copies.
+    const int col0 = h * D;
+    const int qrow = t * p.P + row0;
+    if (elect_one()) {
       mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * Cf::kTileBytes);
 #pragma unroll
       for (int c = 0; c < Cf::kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &p.tm_q, bar_q, col0 + c * 64, qrow, b);
@@ -312,133 +322,154 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         for (int c = 0; c < Cf::kChunks; ++c)
           tma_load_3d(sQ + Cf::kTileBytes + c * kChunkBytes, &p.tm_q, bar_q, col0 + c * 64, qrow + kBM, b);
       }
-      int issued = 0;
-      bool ok = true;
-      auto load = [&](const CUtensorMap* tm, int tok) {
-        const int slot = issued % Cf::kSlots;
-        const uint32_t phase = (issued / Cf::kSlots) & 1;
-        if (!wait_bounded(bar_empty + slot, phase ^ 1, w)) {
-          ok = false;
-          return;
-        }
+    }
+    __syncwarp();
+    int issued = 0;
+    bool ok = true;
+    auto load = [&](const CUtensorMap* tm, int tok) {
+      const int slot = issued % Cf::kSlots;
+      const uint32_t phase = (issued / Cf::kSlots) & 1;
+      if (!__all_sync(0xffffffffu, wait_bounded(bar_empty + slot, phase ^ 1, w))) {
+        ok = false;
+        return;
+      }
+      if (elect_one()) {
         mbar_arrive_expect_tx(bar_full + slot, Cf::kTileBytes);
         uint8_t* dst = sRing + slot * Cf::kTileBytes;
 #pragma unroll
-        for (int c = 0; c < Cf::kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, tm, bar_full + slot, col0 + c * 64, tok, b);
-        ++issued;
-      };
-      // consumption order of the MMA warp: K0, V0, K1, V1, ...
-      TileWalk walk(list, p.L, p.T, p.P);
-      int tok, nv;
-      while (ok && walk.next(tok, nv)) {
-        load(&p.tm_k, tok);
-        if (ok) load(&p.tm_v, tok);
+        for (int c = 0; c < Cf::kChunks; ++c)
+          tma_load_3d(dst + c * kChunkBytes, tm, bar_full + slot, col0 + c * 64, tok, b);
       }
-      if (walk.bad) atomicOr(&g_lvsa_dev_status, LVSA_DEV_BAD_LIST);
-      if (!ok) {
-        // stopped early: let every copy still in flight land before the CTA exits
-        wait_drain(bar_q, 0, p.wait_ns);
-        const int first = issued > Cf::kSlots ? issued - Cf::kSlots : 0;
-        for (int i = first; i < issued; ++i) wait_drain(bar_full + i % Cf::kSlots, (i / Cf::kSlots) & 1, p.wait_ns);
-      }
+      __syncwarp();
+      ++issued;
+    };
+    // consumption order of the MMA warp: K0, V0, K1, V1, ...
+    TileWalk walk(list, p.L, p.T, p.P);
+    int tok, nv;
+    while (ok && walk.next(tok, nv)) {
+      load(&p.tm_k, tok);
+      if (ok) load(&p.tm_v, tok);
+    }
+    if (walk.bad && lane == 0) atomicOr(&g_lvsa_dev_status, LVSA_DEV_BAD_LIST);
+    if (!ok) {
+      // stopped early: let every copy still in flight land before the CTA exits
+      wait_drain(bar_q, 0, p.wait_cycles);
+      const int first = issued > Cf::kSlots ? issued - Cf::kSlots : 0;
+      for (int i = first; i < issued; ++i) wait_drain(bar_full + i % Cf::kSlots, (i / Cf::kSlots) & 1, p.wait_cycles);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // Per K/V tile j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while softmax 1 works on S_1(j)
-    // the tensor core runs tile 0's products, and the other way round.
-    if (lane == 0) {
-      const uint32_t sq = smem_u32(sQ);
-      const uint32_t sr = smem_u32(sRing);
-      const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
-      auto qk = [&](int i, uint32_t k_addr, int n_mma) {
-        const uint32_t q_addr = sq + i * Cf::kTileBytes;
-        const uint32_t idesc = idesc_bf16_f32(kBM, n_mma, false);
+    // the tensor core runs tile 0's products, and the other way round.  The whole warp
+    // runs the schedule (descriptors stay warp-uniform); one elected lane issues.
+    const uint32_t sq = smem_u32(sQ);
+    const uint32_t sr = smem_u32(sRing);
+    const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+    // descriptor of a K-major Q/K tile at byte address a; + (kk>>2)*16 KB + (kk&3)*32 B per 16-wide k-step
+    const uint64_t kdesc0 = smem_desc_sw128(0, 16, 1024);
+    // descriptor of an MN-major V tile: 64-wide d chunks 16 KB apart (LBO), 8-key groups 1 KB apart (SBO)
+    const uint64_t vdesc0 = smem_desc_sw128(0, kChunkBytes, 1024);
+    auto qk = [&](int i, uint32_t k_addr, int n_mma) {
+      const uint64_t qd = kdesc0 + ((sq + i * Cf::kTileBytes) >> 4);
+      const uint64_t kd = kdesc0 + (k_addr >> 4);
+      const uint32_t idesc = idesc_bf16_f32(kBM, n_mma, false);
+      const bool leader = elect_one();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // A = Q, B = K, both K-major: 16-element (32-byte) steps inside a 128-byte swizzle row
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          mma_ss(tmem + 128 * i, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024),
-                 idesc, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate) {
-        for (int kk = 0; kk < n_mma / 16; ++kk) {
-          // B = V tile, MN-major (d contiguous): 64-wide d chunks 16 KB apart (LBO), 8-key groups 1 KB apart (SBO)
-          const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 16 * 128, kChunkBytes, 1024);
-          mma_ts(tmem + kOCol0 + 128 * i, tmem + 128 * i + kk * 8, bdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
-        }
-      };
-      auto slot_of = [&](int idx) { return idx % Cf::kSlots; };
-      auto wait_full = [&](int idx) { return wait_bounded(bar_full + slot_of(idx), (idx / Cf::kSlots) & 1, w); };
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+        if (leader) mma_ss(tmem + 128 * i, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate) {
+      const uint64_t vd = vdesc0 + (v_addr >> 4);
+      const bool leader = elect_one();
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        if (kk * 16 >= n_mma) break;
+        if (leader)
+          mma_ts(tmem + kOCol0 + 128 * i, tmem + 128 * i + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
+                 (accumulate || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) mma_commit(bar);
+      __syncwarp();
+    };
+    auto slot_of = [&](int idx) { return idx % Cf::kSlots; };
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_bounded(bar, parity, w));
+    };
+    auto wait_full = [&](int idx) { return wait_all(bar_full + slot_of(idx), (idx / Cf::kSlots) & 1); };
 
-      int cidx = 0;
-      bool ok = wait_bounded(bar_q, 0, w);
-      TileWalk walk(list, p.L, p.T, p.P);
-      int tok, nv;
-      if (ok && walk.next(tok, nv)) {
-        int n_cur = (nv + 15) & ~15;
-        const int k0 = cidx++;
-        ok = wait_full(k0);
-        if (ok) {
-          tc_fence_after();
-          const uint32_t k_addr = sr + slot_of(k0) * Cf::kTileBytes;
-          qk(0, k_addr, n_cur);
-          mma_commit(bar_s + 0);
-          if (has1) {
-            qk(1, k_addr, n_cur);
-            mma_commit(bar_s + 1);
-          }
-          mma_commit(bar_empty + slot_of(k0));
+    int cidx = 0;
+    bool ok = wait_all(bar_q, 0);
+    TileWalk walk(list, p.L, p.T, p.P);
+    int tok, nv;
+    if (ok && walk.next(tok, nv)) {
+      int n_cur = (nv + 15) & ~15;
+      const int k0 = cidx++;
+      ok = wait_full(k0);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t k_addr = sr + slot_of(k0) * Cf::kTileBytes;
+        qk(0, k_addr, n_cur);
+        commit(bar_s + 0);
+        if (has1) {
+          qk(1, k_addr, n_cur);
+          commit(bar_s + 1);
         }
-        for (int j = 0; ok; ++j) {
-          int tok_n, nv_n;
-          const bool has_next = walk.next(tok_n, nv_n);
-          const int n_next = (nv_n + 15) & ~15;
-          const int vi = cidx++;
-          const uint32_t v_addr = sr + slot_of(vi) * Cf::kTileBytes;
-          if (!wait_bounded(bar_p + 0, j & 1, w) || !wait_full(vi)) {
+        commit(bar_empty + slot_of(k0));
+      }
+      for (int j = 0; ok; ++j) {
+        int tok_n, nv_n;
+        const bool has_next = walk.next(tok_n, nv_n);
+        const int n_next = (nv_n + 15) & ~15;
+        const int vi = cidx++;
+        const uint32_t v_addr = sr + slot_of(vi) * Cf::kTileBytes;
+        if (!wait_all(bar_p + 0, j & 1) || !wait_full(vi)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        pv(0, v_addr, n_cur, j > 0);
+        commit(bar_o + 0);
+        int ki = -1;
+        uint32_t k_addr = 0;
+        if (has_next) {
+          ki = cidx++;
+          k_addr = sr + slot_of(ki) * Cf::kTileBytes;
+          if (!wait_full(ki)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          pv(0, v_addr, n_cur, j > 0);
-          mma_commit(bar_o + 0);
-          int ki = -1;
-          uint32_t k_addr = 0;
-          if (has_next) {
-            ki = cidx++;
-            k_addr = sr + slot_of(ki) * Cf::kTileBytes;
-            if (!wait_full(ki)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            qk(0, k_addr, n_next);
-            mma_commit(bar_s + 0);
-          }
-          if (has1) {
-            if (!wait_bounded(bar_p + 1, j & 1, w)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            pv(1, v_addr, n_cur, j > 0);
-            mma_commit(bar_o + 1);
-          }
-          mma_commit(bar_empty + slot_of(vi));
-          if (!has_next) break;
-          if (has1) {
-            qk(1, k_addr, n_next);
-            mma_commit(bar_s + 1);
-          }
-          mma_commit(bar_empty + slot_of(ki));
-          n_cur = n_next;
+          qk(0, k_addr, n_next);
+          commit(bar_s + 0);
         }
+        if (has1) {
+          if (!wait_all(bar_p + 1, j & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv(1, v_addr, n_cur, j > 0);
+          commit(bar_o + 1);
+        }
+        commit(bar_empty + slot_of(vi));
+        if (!has_next) break;
+        if (has1) {
+          qk(1, k_addr, n_next);
+          commit(bar_s + 1);
+        }
+        commit(bar_empty + slot_of(ki));
+        n_cur = n_next;
       }
-      // every MMA issued must be complete before TMEM is released
-      mma_commit(bar_drain);
-      wait_drain(bar_drain, 0, p.wait_ns);
     }
+    // every MMA issued must be complete before TMEM is released
+    commit(bar_drain);
+    wait_drain(bar_drain, 0, p.wait_cycles);
     __syncwarp();
   }
   } else {
@@ -506,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
 }
 
 // One CTA waits on a barrier that nothing arrives on; the bounded wait runs out.
-__global__ void watchdog_selftest_kernel(unsigned long long budget_ns) {
+__global__ void watchdog_selftest_kernel(long long budget_cycles) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -515,7 +546,7 @@ __global__ void watchdog_selftest_kernel(unsigned long long budget_ns) {
     fence_barrier_init();
   }
   __syncthreads();
-  const Watch w{budget_ns, &abort_flag};
+  const Watch w{budget_cycles, &abort_flag};
   (void)__all_sync(0xffffffffu, wait_bounded(&bar, 0, w));
 }
 
@@ -629,7 +660,7 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   kp.qblocks = qblocks;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   kp.scale_log2 = sc * 1.4426950408889634f;
-  kp.wait_ns = g_wait_ns;
+  kp.wait_cycles = static_cast<long long>(static_cast<double>(g_wait_ns) * kBudgetCyclesPerNs);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch<128>(kp, batch, st, dev) : launch<64>(kp, batch, st, dev);
 }
@@ -655,7 +686,8 @@ extern "C" lvsa_status lvsa_set_wait_budget_ns(unsigned long long ns) {
 extern "C" lvsa_status lvsa_watchdog_selftest(unsigned long long budget_ns, void* stream) {
   if (budget_ns < 1000ull) budget_ns = 1000ull;
   if (budget_ns > 10000000000ull) return LVSA_ERR_INVALID_ARG;
-  lvsa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_ns);
+  lvsa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<long long>(static_cast<double>(budget_ns) * lvsa::kBudgetCyclesPerNs));
   return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
 }
 
