@@ -55,6 +55,9 @@ constexpr int kChunkBytes = kBM * 128;    // one 128-byte-wide swizzle column of
 constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the max grows by > 2^8
 constexpr int kPolyEvery = 0;             // every kPolyEvery-th element pair takes the FMA-pipe exp2 (0: none)
 
+constexpr int kMaxT = 4096;               // latent frames supported (frame bitmaps in shared memory)
+constexpr int kMapWords = kMaxT / 32;
+
 template <int D>
 struct Cfg {
   static constexpr int kChunks = D / 64;
@@ -64,7 +67,8 @@ struct Cfg {
   static constexpr int kOffRing = kQTiles * kTileBytes;
   static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
   static constexpr int kBarBytes = 512;
-  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
+  static constexpr int kOffMap = kOffBar + kBarBytes;             // two frame bitmaps of kMapWords words
+  static constexpr int kSmemBytes = kOffMap + 2 * kMapWords * 4 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(8 * (1 + 2 * kSlots + 7) + 8 <= kBarBytes, "barrier area");
 };
@@ -76,7 +80,9 @@ struct KernelParams {
   __nv_bfloat16* out;
   const int32_t* lists;
   int T, P, H, L;
-  int qblocks;       // ceil(P / 256): CTAs per query frame
+  int straddle;      // 1: CTA c takes query rows [256c, 256c+256) of the whole frame-major sequence
+  int qblocks;       // straddle == 0: ceil(P / 256) CTAs per query frame
+  int nblocks;       // CTAs per (batch, head)
   float scale_log2;  // softmax scale * log2(e)
   long long wait_cycles;
 };
@@ -123,37 +129,53 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long 
 }
 
 // ------------------------------------------------------------------ K/V tile walk
-// Walks the frame list of one query frame as runs of consecutive frames and
-// cuts each run's token range into tiles of at most 128 tokens.  Every role
-// of the CTA walks the same sequence.
-struct TileWalk {
-  const int32_t* list;
-  int L, T, P;
-  int li = 0, pos = 0, end = 0;
-  bool bad = false;
+// The CTA's query rows belong to frame fa, or to frames fa and fb = fa + 1.  Their
+// frame lists are held as bitmaps over [0, T) (so list order and duplicates do not
+// matter).  The walk visits the union in ascending frame order as runs of
+// consecutive frames with the same membership (bit 0: attended by fa, bit 1: by
+// fb); a run is one contiguous token range, cut into tiles of at most 128 tokens.
+// Every role of the CTA walks the same sequence.
+struct FrameWalk {
+  const uint32_t* ma;
+  const uint32_t* mb;
+  int T, P, nwords;
+  int f = 0, pos = 0, end = 0, mask = 0;
 
-  __device__ TileWalk(const int32_t* l, int L_, int T_, int P_) : list(l), L(L_), T(T_), P(P_) {}
+  __device__ FrameWalk(const uint32_t* a, const uint32_t* b_, int T_, int P_)
+      : ma(a), mb(b_), T(T_), P(P_), nwords((T_ + 31) >> 5) {}
 
-  __device__ __forceinline__ bool next(int& tok, int& nvalid) {
+  __device__ __forceinline__ int bits(int g) const {
+    return static_cast<int>(((ma[g >> 5] >> (g & 31)) & 1u) | (((mb[g >> 5] >> (g & 31)) & 1u) << 1));
+  }
+
+  __device__ __forceinline__ bool next(int& tok, int& nvalid, int& tmask) {
     while (pos >= end) {
-      if (li >= L) return false;
-      const int f0 = __ldg(list + li++);
-      if (f0 < 0 || f0 >= T) {
-        bad = true;
-        continue;
+      if (f >= T) return false;
+      int wi = f >> 5;
+      uint32_t word = (ma[wi] | mb[wi]) & (0xffffffffu << (f & 31));
+      while (word == 0) {
+        if (++wi >= nwords) {
+          f = T;
+          return false;
+        }
+        word = ma[wi] | mb[wi];
       }
+      const int f0 = (wi << 5) + __ffs(word) - 1;
+      if (f0 >= T) {
+        f = T;
+        return false;
+      }
+      const int m0 = bits(f0);
       int f1 = f0;
-      while (li < L) {
-        const int f = __ldg(list + li);
-        if (f != f1 + 1 || f >= T) break;
-        f1 = f;
-        ++li;
-      }
+      while (f1 + 1 < T && bits(f1 + 1) == m0) ++f1;
       pos = f0 * P;
       end = (f1 + 1) * P;
+      mask = m0;
+      f = f1 + 1;
     }
     tok = pos;
     nvalid = min(kBN, end - pos);
+    tmask = mask;
     pos += nvalid;
     return true;
   }
@@ -163,10 +185,11 @@ struct TileWalk {
 // Thread = one query row.  Loads the row of S from TMEM, masks columns past the
 // run end, updates the running max lazily (rescaling the row of O in TMEM when
 // needed), writes P = 2^(scale*log2e*s - m) as bf16 over the S columns and
-// returns the row sum of P through `l`.
+// returns the row sum of P through `l`.  `skip`: the row's frame does not attend
+// the tile (P = 0, max and sum unchanged).
 template <int D>
-__device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int nv, int j, float sl2, float& m,
-                                             float& l, uint64_t* bar_o, const Watch& w) {
+__device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int nv, int j, bool skip, float sl2,
+                                             float& m, float& l, uint64_t* bar_o, const Watch& w) {
   float s[kBN];
   tmem_ld32(s_tmem + 0, s + 0);
   if (nv > 32) tmem_ld32(s_tmem + 32, s + 32);
@@ -193,7 +216,10 @@ __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[120 + k]);
-  const float tile_max = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7])) * sl2;
+  // a row whose frame does not attend this tile's frames takes no part in it:
+  // its max stays and its P is 2^-inf = 0
+  const float tile_max =
+      skip ? -INFINITY : fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7])) * sl2;
 
   float alpha = 1.f;
   if (tile_max > m + kRescaleLog2) {
@@ -217,7 +243,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
   }
 
   const float2 scale2 = make_float2(sl2, sl2);
-  const float2 negm2 = make_float2(-m, -m);
+  const float2 negm2 = skip ? make_float2(-INFINITY, -INFINITY) : make_float2(-m, -m);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -267,13 +293,47 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qb = blockIdx.x % p.qblocks;
-  const int t = blockIdx.x / p.qblocks;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
-  const int row0 = qb * kQTiles * kBM;        // first query row (within frame t) of this CTA
-  const bool has1 = row0 + kBM < p.P;         // the second query tile has rows
-  const int32_t* list = p.lists + static_cast<size_t>(t) * p.L;
+  const int ltok = p.T * p.P;
+  // query rows [r0, r1) of the frame-major sequence: one frame fa, or fa and fb = fa + 1
+  int r0, r1;
+  if (p.straddle) {
+    r0 = blockIdx.x * (kQTiles * kBM);
+    r1 = min(r0 + kQTiles * kBM, ltok);
+  } else {
+    const int qb = blockIdx.x % p.qblocks;
+    const int t = blockIdx.x / p.qblocks;
+    r0 = t * p.P + qb * (kQTiles * kBM);
+    r1 = min(r0 + kQTiles * kBM, (t + 1) * p.P);
+  }
+  const int fa = r0 / p.P;
+  const int fb = (r1 - 1) / p.P;
+  const bool has1 = r0 + kBM < r1;  // the second query tile has rows
+  uint32_t* map_a = reinterpret_cast<uint32_t*>(smem + Cf::kOffMap);
+  uint32_t* map_b = map_a + kMapWords;
+  {
+    // frame bitmaps of the lists of fa and fb (map_b stays empty when fb == fa)
+    const int nwords = (p.T + 31) >> 5;
+    for (int i = threadIdx.x; i < nwords; i += kThreads) {
+      map_a[i] = 0u;
+      map_b[i] = 0u;
+    }
+    __syncthreads();
+    bool bad = false;
+    const int32_t* la = p.lists + static_cast<size_t>(fa) * p.L;
+    const int32_t* lb = p.lists + static_cast<size_t>(fb) * p.L;
+    const int nset = (fb != fa) ? 2 * p.L : p.L;
+    for (int i = threadIdx.x; i < nset; i += kThreads) {
+      const int f = (i < p.L) ? __ldg(la + i) : __ldg(lb + (i - p.L));
+      if (f < 0 || f >= p.T) {
+        bad = true;
+        continue;
+      }
+      atomicOr((i < p.L ? map_a : map_b) + (f >> 5), 1u << (f & 31));
+    }
+    if (bad) atomicOr(&g_lvsa_dev_status, LVSA_DEV_BAD_LIST);
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -312,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     // The whole warp walks the list (warp-uniform control flow); one elected
     // lane arms the barriers and issues the copies.
     const int col0 = h * D;
-    const int qrow = t * p.P + row0;
+    const int qrow = r0;
     if (elect_one()) {
       mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * Cf::kTileBytes);
 #pragma unroll
@@ -344,13 +404,12 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       ++issued;
     };
     // consumption order of the MMA warp: K0, V0, K1, V1, ...
-    TileWalk walk(list, p.L, p.T, p.P);
-    int tok, nv;
-    while (ok && walk.next(tok, nv)) {
+    FrameWalk walk(map_a, map_b, p.T, p.P);
+    int tok, nv, tmask;
+    while (ok && walk.next(tok, nv, tmask)) {
       load(&p.tm_k, tok);
       if (ok) load(&p.tm_v, tok);
     }
-    if (walk.bad && lane == 0) atomicOr(&g_lvsa_dev_status, LVSA_DEV_BAD_LIST);
     if (!ok) {
       // stopped early: let every copy still in flight land before the CTA exits
       wait_drain(bar_q, 0, p.wait_cycles);
@@ -405,9 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
 
     int cidx = 0;
     bool ok = wait_all(bar_q, 0);
-    TileWalk walk(list, p.L, p.T, p.P);
-    int tok, nv;
-    if (ok && walk.next(tok, nv)) {
+    FrameWalk walk(map_a, map_b, p.T, p.P);
+    int tok, nv, tmask;
+    if (ok && walk.next(tok, nv, tmask)) {
       int n_cur = (nv + 15) & ~15;
       const int k0 = cidx++;
       ok = wait_full(k0);
@@ -423,8 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         commit(bar_empty + slot_of(k0));
       }
       for (int j = 0; ok; ++j) {
-        int tok_n, nv_n;
-        const bool has_next = walk.next(tok_n, nv_n);
+        int tok_n, nv_n, tmask_n;
+        const bool has_next = walk.next(tok_n, nv_n, tmask_n);
         const int n_next = (nv_n + 15) & ~15;
         const int vi = cidx++;
         const uint32_t v_addr = sr + slot_of(vi) * Cf::kTileBytes;
@@ -485,13 +544,15 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       float l = 0.f;        // running sum of 2^(scaled s - m)
       bool ok = true;
       int j = 0;
-      TileWalk walk(list, p.L, p.T, p.P);
-      int tok, nv;
-      while (walk.next(tok, nv)) {
+      const int row = r0 + qi * kBM + r;  // query row in the frame-major sequence
+      const int rbit = (row / p.P == fa) ? 1 : 2;
+      FrameWalk walk(map_a, map_b, p.T, p.P);
+      int tok, nv, tmask;
+      while (walk.next(tok, nv, tmask)) {
         ok = __all_sync(0xffffffffu, wait_bounded(bar_s + qi, j & 1, w));
         if (!ok) break;
         tc_fence_after();
-        ok = softmax_tile<D>(s_tmem, o_tmem, nv, j, p.scale_log2, m, l, bar_o + qi, w);
+        ok = softmax_tile<D>(s_tmem, o_tmem, nv, j, (tmask & rbit) == 0, p.scale_log2, m, l, bar_o + qi, w);
         if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
@@ -502,12 +563,9 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         ok = __all_sync(0xffffffffu, wait_bounded(bar_o + qi, (j - 1) & 1, w));
         if (ok) {
           tc_fence_after();
-          const float inv_l = 1.f / l;
-          const int row = row0 + qi * kBM + r;
-          const bool valid = row < p.P;
-          const size_t ltok = static_cast<size_t>(p.T) * p.P;
-          __nv_bfloat16* dst =
-              p.out + ((static_cast<size_t>(b) * ltok + static_cast<size_t>(t) * p.P + row) * p.H + h) * D;
+          const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a frame with no valid list entry: zero output
+          const bool valid = row < r1;
+          __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * ltok + row) * p.H + h) * D;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
@@ -612,7 +670,7 @@ lvsa_status launch(const KernelParams& kp, int B, cudaStream_t stream, int dev) 
       g_attr_set[di][dev] = true;
     }
   }
-  dim3 grid(static_cast<unsigned>(kp.T * kp.qblocks), static_cast<unsigned>(kp.H), static_cast<unsigned>(B));
+  dim3 grid(static_cast<unsigned>(kp.nblocks), static_cast<unsigned>(kp.H), static_cast<unsigned>(B));
   lvsa_attention_kernel<D><<<grid, kThreads, Cf::kSmemBytes, stream>>>(kp);
   return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
 }
@@ -637,8 +695,15 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lists) & 3u))
     return LVSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return LVSA_ERR_UNSUPPORTED;
+  if (T > kMaxT) return LVSA_ERR_UNSUPPORTED;
   const int qblocks = (P + kQTiles * kBM - 1) / (kQTiles * kBM);
-  if (static_cast<long long>(T) * qblocks > INT_MAX) return LVSA_ERR_INVALID_ARG;
+  // frames of at least 256 tokens: query blocks of 256 rows run over the whole
+  // sequence (a block may hold the end of one frame and the start of the next);
+  // shorter frames: blocks stay inside a frame
+  const int straddle = P >= kQTiles * kBM ? 1 : 0;
+  const long long nblocks = straddle ? (static_cast<long long>(T) * P + kQTiles * kBM - 1) / (kQTiles * kBM)
+                                     : static_cast<long long>(T) * qblocks;
+  if (nblocks > INT_MAX) return LVSA_ERR_INVALID_ARG;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LVSA_ERR_CUDA;
@@ -658,6 +723,8 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   kp.H = heads;
   kp.L = L;
   kp.qblocks = qblocks;
+  kp.straddle = straddle;
+  kp.nblocks = static_cast<int>(nblocks);
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   kp.scale_log2 = sc * 1.4426950408889634f;
   kp.wait_cycles = static_cast<long long>(static_cast<double>(g_wait_ns) * kBudgetCyclesPerNs);

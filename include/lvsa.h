@@ -102,12 +102,12 @@ lvsa_status lvsa_build_anchors(int T, int C, int W, long long step,
  *            aligned.  Values must be finite.
  *   lists    DEVICE int32 [T][L], row t = the frames attended by query frame t
  *            (as written by lvsa_build_frame_lists, or 0..T-1 in every row for
- *            dense attention).  Rows should be ascending without duplicates:
- *            runs of consecutive frames are fetched as one token range, a
- *            duplicated frame is attended twice.  Entries outside [0,T) are
- *            skipped and flag LVSA_DEV_BAD_LIST.
+ *            dense attention).  A row is a set: order and repeated entries do
+ *            not matter.  Entries outside [0,T) are skipped and flag
+ *            LVSA_DEV_BAD_LIST; a frame with no valid entry gets a zero output.
  *   L        list width, 1 <= L <= T.
- *   T, tokens_per_frame (P), heads (H), d, batch: sizes; d must be 64 or 128.
+ *   T, tokens_per_frame (P), heads (H), d, batch: sizes; d must be 64 or 128;
+ *            T <= 4096 (LVSA_ERR_UNSUPPORTED above).
  *   scale    softmax scale; <= 0 selects 1/sqrt(d).
  *   out      DEVICE bf16, same layout as q, 16-byte aligned, must not alias
  *            q, k or v.

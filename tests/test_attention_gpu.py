@@ -199,3 +199,32 @@ def test_fma_pipe_exp2_against_cuda_exp2(gpu_lib):
     rel = ((y.double() - ref).abs() / ref).max().item()
     assert rel <= 1e-4, rel
     assert (y > 0).all() and torch.isfinite(y).all()
+
+
+@pytest.mark.parametrize("T,P,d", [(10, 300, 128), (6, 200, 64), (9, 517, 128)])
+def test_random_lists_are_sets(gpu_lib, T, P, d):
+    # arbitrary per-frame lists, unsorted and with duplicates: each row is the set of its
+    # frames; query blocks that straddle two frames attend the union with per-row masks
+    g = np.random.default_rng(T * P)
+    L = 5
+    lists = g.integers(0, T, size=(T, L)).astype(np.int32)
+    lists[1, :] = lists[1, 0]                    # one frame listed L times
+    q, k, v = make(T, P, 2, d, seed=P)
+    out = full_out(run_kernel(gpu_lib, q, k, v, lists, P))
+    ref = OA.sparse_attention(q, k, v, [sorted(set(int(f) for f in r)) for r in lists], P)
+    assert_close(out, ref, "random set lists")
+
+
+def test_frame_without_valid_entries_gives_zeros(gpu_lib):
+    T, P, H, d = 7, 300, 2, 128
+    q, k, v = make(T, P, H, d, seed=21)
+    gpu_lib.lvsa_get_device_status(clear=True)
+    lists = gpu_lib.lvsa_build_frame_lists(T, 3, 1, 1).copy()
+    lists[4, :] = -1
+    out = full_out(run_kernel(gpu_lib, q, k, v, lists, P))
+    assert gpu_lib.lvsa_get_device_status(clear=True) & gpu_lib.LVSA_DEV_BAD_LIST
+    assert np.all(out[:, 4 * P:5 * P] == 0)
+    good = [list(r) for r in lists]
+    rows = [r for r in range(T * P) if r // P != 4]
+    ref = OA.sparse_attention_rows(q, k, v, good, P, rows)
+    assert_close(out[:, rows], ref, "other frames")
