@@ -230,8 +230,8 @@ def run_reference(args, rank, world):
     return 0
 
 
-def workload_config(w, world):
-    return {"workload": w.name, "T": w.T, "tokens_per_frame": w.P, "heads": w.H, "head_dim": w.d, "C": w.C,
+def workload_config(w, world, fixed_grid=False):
+    return {"workload": w.name, "anchors": "fixed grid (step 0 pattern every step)" if fixed_grid else "rotating", "T": w.T, "tokens_per_frame": w.P, "heads": w.H, "head_dim": w.d, "C": w.C,
             "W": w.W, "G": max(0, w.C - w.W) if w.C < w.T else 0, "global_batch": w.B * world,
             "seq_len": w.T * w.P, "parallelism": "replicas" if world > 1 else "single",
             "l2": "inputs larger than L2 (Q+K+V+O working set "
@@ -258,9 +258,13 @@ def run_lvsa(args, rank, world, local):
     lists_dev = torch.empty((w.T, w.L), dtype=torch.int32, device=dev)
     build_us = []
 
+    def list_step(s):
+        # fixed-grid ablation: the anchors never rotate, i.e. the step-0 pattern at every step
+        return 0 if args.fixed_grid else s
+
     def step(s, host_list_buf):
         t0 = time.perf_counter()
-        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=host_list_buf.numpy())
+        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, list_step(s), out=host_list_buf.numpy())
         build_us.append((time.perf_counter() - t0) * 1e6)
         lists_dev.copy_(host_list_buf, non_blocking=True)
         lvsa.lvsa_attention(q, k, v, lists_dev, w.P, out=out, stream=stream)
@@ -279,7 +283,7 @@ def run_lvsa(args, rank, world, local):
         for i in range(args.steps):
             s = args.warmup + i
             t0 = time.perf_counter()
-            lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=pinned[s].numpy())
+            lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, list_step(s), out=pinned[s].numpy())
             build_us.append((time.perf_counter() - t0) * 1e6)
             lists_dev.copy_(pinned[s], non_blocking=True)
             ev_k[i][0].record(stream)
@@ -327,7 +331,7 @@ def run_lvsa(args, rank, world, local):
         q.copy_(qh, non_blocking=True)
         k.copy_(kh, non_blocking=True)
         v.copy_(vh, non_blocking=True)
-        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=pinned[s % nsteps].numpy())
+        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, list_step(s), out=pinned[s % nsteps].numpy())
         lists_dev.copy_(pinned[s % nsteps], non_blocking=True)
         lvsa.lvsa_attention(q, k, v, lists_dev, w.P, out=out, stream=stream)
         oh.copy_(out, non_blocking=True)
@@ -365,7 +369,7 @@ def run_lvsa(args, rank, world, local):
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, world),
+        "config": workload_config(w, world, args.fixed_grid),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 dense (burst)",
@@ -386,6 +390,48 @@ def run_lvsa(args, rank, world, local):
                                           f"{t:.1f} s of fp64 numpy on the host"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_sweep(args, rank, world, local):
+    """Horizon sweep at the Wan-1.3B budget (C = 21, W = 9, H = 12, P = 1560): the same kernel with the
+    LVSA lists and with dense lists (C = T) for T = 21 ... 257 latent frames; one JSON line per T."""
+    import torch
+
+    import block_sparse_attention_frame_b200 as lvsa
+    from block_sparse_attention_frame_b200 import synthetic
+
+    if rank != 0:
+        return 0
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    base = synthetic.WORKLOADS["wan1.3b_6x"]
+    for T in [int(x) for x in args.sweep_T.split(",")]:
+        w = synthetic.Workload(f"wan1.3b_T{T}", T=T, P=base.P, H=base.H, d=base.d, C=base.C, W=base.W, seed=2000 + T)
+        q, k, v = synthetic.make_qkv(w, device=dev)
+        out = torch.empty_like(q)
+        res = {}
+        for kind, C in (("sparse", w.C), ("dense", T)):
+            lists = torch.from_numpy(lvsa.lvsa_build_frame_lists(T, C, min(w.W, C), 7)).to(dev)
+            calls = 3 if kind == "sparse" or T <= 121 else 1
+            for _ in range(2):
+                lvsa.lvsa_attention(q, k, v, lists, w.P, out=out)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(calls):
+                lvsa.lvsa_attention(q, k, v, lists, w.P, out=out)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / calls
+            L = lists.shape[1]
+            res[kind] = (ms, 4.0 * w.B * w.H * T * L * w.P * w.P * w.d / (ms * 1e-3) / 1e12)
+        print(json.dumps({"sweep": "horizon", "T": T, "video_frames": 4 * (T - 1) + 1, "C": w.C, "W": w.W,
+                          "sparse_ms": res["sparse"][0], "sparse_tflops": res["sparse"][1],
+                          "dense_ms": res["dense"][0], "dense_tflops": res["dense"][1],
+                          "speedup": res["dense"][0] / res["sparse"][0]}), flush=True)
+        del q, k, v, out
+        torch.cuda.empty_cache()
     return 0
 
 
@@ -412,6 +458,11 @@ def main(argv=None):
     ap.add_argument("--impl", default="lvsa", choices=["lvsa", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fixed-grid", action="store_true",
+                    help="ablation: anchors do not rotate (the step-0 pattern at every step)")
+    ap.add_argument("--sweep", choices=["horizon"], default=None,
+                    help="horizon sweep: sparse vs dense for several T (one JSON line per T)")
+    ap.add_argument("--sweep-T", default="21,41,81,121,161,257")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device path only and print a short line (for profiling runs)")
     ap.add_argument("--ref-seconds", type=float, default=0.0, help="reference arm: CPU seconds per step")
@@ -421,6 +472,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.sweep:
+            return run_sweep(args, rank, world, local)
         return run_lvsa(args, rank, world, local)
     finally:
         if world > 1:

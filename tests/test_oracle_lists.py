@@ -209,3 +209,17 @@ def test_mistake_window_not_shifted_is_caught(monkeypatch):
     monkeypatch.setattr(OL, "window", unshifted)
     with pytest.raises(AssertionError):
         test_invariants_brute_force()
+
+
+def test_fixed_grid_ablation_never_covers_intermediate_frames():
+    # the non-rotating pattern the pages contrast with (gist.science summary, "Rotating Global
+    # Anchors": a fixed grid leaves intermediate frames seen only locally): holding the step at 0,
+    # only the G grid frames are ever anchors; with rotation every frame is, within T_per steps
+    T, C, W = 121, 21, 9
+    G, Tper = C - W, OL.anchor_period(T, C, W)
+    fixed = [0] * T
+    for _ in range(Tper):
+        for f in OL.anchors(T, C, W, 0):
+            fixed[f] += 1
+    assert sum(1 for c in fixed if c == 0) == T - G
+    assert min(OL.anchor_coverage(T, C, W, 0)) >= 1
