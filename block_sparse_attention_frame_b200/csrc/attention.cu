@@ -70,7 +70,7 @@ struct Cfg {
   static constexpr int kOffMap = kOffBar + kBarBytes;             // two frame bitmaps of kMapWords words
   static constexpr int kSmemBytes = kOffMap + 2 * kMapWords * 4 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert(8 * (1 + 2 * kSlots + 7) + 8 <= kBarBytes, "barrier area");
+  static_assert(8 * (1 + 2 * kSlots + 9) + 8 <= kBarBytes, "barrier area");
 };
 
 struct KernelParams {
@@ -186,10 +186,12 @@ struct FrameWalk {
 // run end, updates the running max lazily (rescaling the row of O in TMEM when
 // needed), writes P = 2^(scale*log2e*s - m) as bf16 over the S columns and
 // returns the row sum of P through `l`.  `skip`: the row's frame does not attend
-// the tile (P = 0, max and sum unchanged).
+// the tile (P = 0, max and sum unchanged).  After the first 64 keys of P are
+// stored it arrives on `bar_half`, so the tensor core can run the first half of
+// PV while this thread computes the second half.
 template <int D>
 __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int nv, int j, bool skip, float sl2,
-                                             float& m, float& l, uint64_t* bar_o, const Watch& w) {
+                                             float& m, float& l, uint64_t* bar_o, const Watch& w, uint64_t* bar_half) {
   float s[kBN];
   tmem_ld32(s_tmem + 0, s + 0);
   if (nv > 32) tmem_ld32(s_tmem + 32, s + 32);
@@ -264,6 +266,12 @@ __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       }
       tmem_st16(s_tmem + 16 * c, pk);  // P overwrites the first half of the S columns
     }
+    if (c == 1) {
+      // keys 0..63 of P are in TMEM: the MMA warp may start the first half of PV
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_half);
+    }
   }
   const float2 t01 = fadd2(acc[0], acc[1]);
   const float2 t23 = fadd2(acc[2], acc[3]);
@@ -287,7 +295,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   uint64_t* bar_s = bar_empty + Cf::kSlots;  // [2] S_i(j) ready in TMEM
   uint64_t* bar_p = bar_s + 2;               // [2] P_i(j) written to TMEM (128 arrivals)
   uint64_t* bar_o = bar_p + 2;               // [2] PV_i(j) finished
-  uint64_t* bar_drain = bar_o + 2;           // all MMAs of the CTA finished
+  uint64_t* bar_ph = bar_o + 2;              // [2] P_i(j) keys 0..63 written (128 arrivals)
+  uint64_t* bar_drain = bar_ph + 2;          // all MMAs of the CTA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -345,6 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       mbar_init(bar_s + i, 1);
       mbar_init(bar_p + i, 4 * 32);
       mbar_init(bar_o + i, 1);
+      mbar_init(bar_ph + i, 4 * 32);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -419,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // Per K/V tile j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while softmax 1 works on S_1(j)
-    // the tensor core runs tile 0's products, and the other way round.  The whole warp
+    // the tensor core runs tile 0's products, and the other way round.  Each PV is issued in two
+    // halves (keys 0..63 as soon as the softmax has stored them, then keys 64..127).  The whole warp
     // runs the schedule (descriptors stay warp-uniform); one elected lane issues.
     const uint32_t sq = smem_u32(sQ);
     const uint32_t sr = smem_u32(sRing);
@@ -440,12 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       }
       __syncwarp();
     };
-    auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate) {
+    auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate, int k_lo, int k_hi) {
       const uint64_t vd = vdesc0 + (v_addr >> 4);
       const bool leader = elect_one();
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk) {
-        if (kk * 16 >= n_mma) break;
+        if (kk < k_lo) continue;
+        if (kk >= k_hi || kk * 16 >= n_mma) break;
         if (leader)
           mma_ts(tmem + kOCol0 + 128 * i, tmem + 128 * i + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
                  (accumulate || kk > 0) ? 1u : 0u);
@@ -487,12 +499,18 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         const int n_next = (nv_n + 15) & ~15;
         const int vi = cidx++;
         const uint32_t v_addr = sr + slot_of(vi) * Cf::kTileBytes;
-        if (!wait_all(bar_p + 0, j & 1) || !wait_full(vi)) {
+        if (!wait_all(bar_ph + 0, j & 1) || !wait_full(vi)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        pv(0, v_addr, n_cur, j > 0);
+        pv(0, v_addr, n_cur, j > 0, 0, 4);
+        if (!wait_all(bar_p + 0, j & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        pv(0, v_addr, n_cur, j > 0, 4, 8);
         commit(bar_o + 0);
         int ki = -1;
         uint32_t k_addr = 0;
@@ -508,12 +526,18 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
           commit(bar_s + 0);
         }
         if (has1) {
+          if (!wait_all(bar_ph + 1, j & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv(1, v_addr, n_cur, j > 0, 0, 4);
           if (!wait_all(bar_p + 1, j & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          pv(1, v_addr, n_cur, j > 0);
+          pv(1, v_addr, n_cur, j > 0, 4, 8);
           commit(bar_o + 1);
         }
         commit(bar_empty + slot_of(vi));
@@ -552,7 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         ok = __all_sync(0xffffffffu, wait_bounded(bar_s + qi, j & 1, w));
         if (!ok) break;
         tc_fence_after();
-        ok = softmax_tile<D>(s_tmem, o_tmem, nv, j, (tmask & rbit) == 0, p.scale_log2, m, l, bar_o + qi, w);
+        ok = softmax_tile<D>(s_tmem, o_tmem, nv, j, (tmask & rbit) == 0, p.scale_log2, m, l, bar_o + qi, w,
+                             bar_ph + qi);
         if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
