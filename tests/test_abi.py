@@ -65,6 +65,7 @@ def test_attention_argument_validation_without_gpu(lib):
     assert call(scale=float("nan")) == INV
     assert call(T=1 << 20, P=1 << 12) == INV  # T*P overflows int32
     assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
+    assert call(T=4097, L=4) == lib.LVSA_ERR_UNSUPPORTED   # frame bitmaps cover up to 4096 latent frames
     # valid arguments on a machine without a B200: a clean error, never a crash
     from conftest import cuda_available
 

@@ -85,6 +85,8 @@ def test_negative_control_wrong_step_fails(gpu_lib):
     (9, 256, 1, 128, 1, 9, 3, 0),     # C = T: dense
     (12, 96, 2, 128, 1, 5, 5, 2),     # G = 0: pure sliding window
     (1, 1000, 2, 128, 1, 21, 9, 0),   # T = 1
+    (5, 300, 2, 128, 2, 3, 1, 2),     # batch 2, 256-row blocks straddling frame boundaries
+    (6, 700, 3, 64, 2, 3, 2, 5),      # batch 2, d = 64, straddling blocks
 ])
 def test_ragged_shapes_full_parity(gpu_lib, T, P, H, d, B, C, W, s):
     q, k, v = make(T, P, H, d, B=B, seed=T * 1000 + P)
