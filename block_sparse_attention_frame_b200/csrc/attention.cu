@@ -117,8 +117,14 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, con
   }
 }
 
-// Used only while shutting down after an abort: ignores the abort flag.
+// Used only while shutting down after an abort: ignores the abort flag.  Copies and
+// MMAs in flight always complete on their own, so the drain allows at least ~1 s
+// whatever the caller's wait budget: a CTA must not exit while a copy can still land
+// in its shared memory.
+constexpr long long kMinDrainCycles = 2000000000ll;
+
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long long budget_cycles) {
+  budget_cycles = budget_cycles > kMinDrainCycles ? budget_cycles : kMinDrainCycles;
   const long long t0 = clock64();
   for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it) {
     if ((it & 63u) == 63u && clock64() - t0 > budget_cycles) {

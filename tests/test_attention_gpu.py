@@ -87,6 +87,9 @@ def test_negative_control_wrong_step_fails(gpu_lib):
     (1, 1000, 2, 128, 1, 21, 9, 0),   # T = 1
     (5, 300, 2, 128, 2, 3, 1, 2),     # batch 2, 256-row blocks straddling frame boundaries
     (6, 700, 3, 64, 2, 3, 2, 5),      # batch 2, d = 64, straddling blocks
+    (7, 1, 2, 64, 1, 3, 1, 4),        # one token per frame
+    (4, 2, 1, 128, 3, 2, 2, 1),       # two tokens per frame, batch 3
+    (9, 130, 1, 128, 1, 1, 1, 0),     # C = W = 1: every frame attends only itself
 ])
 def test_ragged_shapes_full_parity(gpu_lib, T, P, H, d, B, C, W, s):
     q, k, v = make(T, P, H, d, B=B, seed=T * 1000 + P)
