@@ -9,6 +9,8 @@ Functions carry the C ABI's names (declared in ``include/lvsa.h``):
 ``lvsa_build_frame_lists(T, C, W, step)`` -> int32 numpy array [T, min(C,T)]
 ``lvsa_build_anchors(T, C, W, step)``     -> int32 numpy array [G]
 ``lvsa_attention(q, k, v, lists, tokens_per_frame, scale=0, out=None, stream=None)``
+``lvsa_attention_host(q_host, k_host, v_host, lists_host, tokens_per_frame, out_host, q_dev, k_dev, v_dev,
+lists_dev, out_dev, scale=0, heads_per_band=0, stream=None)``
 ``lvsa_get_device_status(clear=False)``   -> int (LVSA_DEV_* bits)
 ``lvsa_set_wait_budget_ns(ns)``, ``lvsa_watchdog_selftest(budget_ns, stream=None)``
 """
@@ -34,7 +36,7 @@ LVSA_DEV_TIMEOUT = 0x1
 LVSA_DEV_BAD_LIST = 0x2
 
 EXPORTED = [
-    "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_get_device_status",
+    "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_attention_host", "lvsa_get_device_status",
     "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_exp2_fma_eval", "lvsa_status_string",
     "lvsa_version",
 ]
@@ -63,6 +65,9 @@ _lib.lvsa_build_anchors.restype = _c_int
 _lib.lvsa_attention.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _c_float, _c_vp, _c_vp]
 _lib.lvsa_attention.restype = _c_int
+_lib.lvsa_attention_host.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                     _c_float, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_vp]
+_lib.lvsa_attention_host.restype = _c_int
 _lib.lvsa_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), _c_int]
 _lib.lvsa_get_device_status.restype = _c_int
 _lib.lvsa_set_wait_budget_ns.argtypes = [_c_ull]
@@ -167,6 +172,53 @@ def lvsa_attention_raw(q_ptr: int, k_ptr: int, v_ptr: int, lists_ptr: int, L: in
     """The C call with raw device pointers; returns the status code unchanged."""
     return int(_lib.lvsa_attention(q_ptr, k_ptr, v_ptr, lists_ptr, L, T, P, H, d, B, float(scale), out_ptr,
                                    ctypes.c_void_p(stream_ptr)))
+
+
+def lvsa_attention_host(q_host, k_host, v_host, lists_host, tokens_per_frame: int, out_host, q_dev, k_dev, v_dev,
+                        lists_dev, out_dev, scale: float = 0.0, heads_per_band: int = 0, stream=None):
+    """Block-sparse attention on host tensors, uploads and readback pipelined by bands of heads.
+
+    q_host, k_host, v_host, out_host: CPU bf16 tensors [batch, T*tokens_per_frame, heads, d], contiguous
+    (pinned for overlap).  lists_host: CPU int32 [T, L].  q_dev, k_dev, v_dev, out_dev, lists_dev: CUDA
+    staging tensors of the same shapes.  Asynchronous on ``stream``: synchronise it before reading out_host.
+    """
+    import torch
+
+    for name, x in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host), ("out_host", out_host)):
+        if not isinstance(x, torch.Tensor) or x.device.type != "cpu" or x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a CPU bfloat16 tensor")
+        if not x.is_contiguous() or x.dim() != 4 or x.shape != q_host.shape:
+            raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q_host")
+    for name, x in (("q_dev", q_dev), ("k_dev", k_dev), ("v_dev", v_dev), ("out_dev", out_dev)):
+        if not isinstance(x, torch.Tensor) or x.device.type != "cuda" or x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+        if not x.is_contiguous() or x.shape != q_host.shape or x.device != q_dev.device:
+            raise ValueError(f"{name} must be contiguous, shaped like q_host, on q_dev's device")
+    if (lists_host.device.type != "cpu" or lists_host.dtype != torch.int32 or lists_host.dim() != 2
+            or not lists_host.is_contiguous()):
+        raise TypeError("lists_host must be a contiguous CPU int32 tensor [T, L]")
+    if (lists_dev.device != q_dev.device or lists_dev.dtype != torch.int32 or lists_dev.shape != lists_host.shape
+            or not lists_dev.is_contiguous()):
+        raise TypeError("lists_dev must be a contiguous CUDA int32 tensor shaped like lists_host")
+    B, ntok, H, d = q_host.shape
+    T, L = lists_host.shape
+    if ntok != T * tokens_per_frame:
+        raise ValueError(f"q_host has {ntok} tokens, expected T*tokens_per_frame = {T * tokens_per_frame}")
+    with torch.cuda.device(q_dev.device):
+        st = _lib.lvsa_attention_host(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), lists_host.data_ptr(),
+                                      L, T, tokens_per_frame, H, d, B, float(scale), out_host.data_ptr(),
+                                      q_dev.data_ptr(), k_dev.data_ptr(), v_dev.data_ptr(), lists_dev.data_ptr(),
+                                      out_dev.data_ptr(), int(heads_per_band), _stream_ptr(stream, q_dev.device))
+    _check("lvsa_attention_host", st)
+    return out_host
+
+
+def lvsa_attention_host_raw(*args) -> int:
+    """The C call with raw pointers (19 arguments in the header's order); returns the status unchanged."""
+    a = list(args)
+    a[10] = float(a[10])
+    a[18] = ctypes.c_void_p(a[18])
+    return int(_lib.lvsa_attention_host(*a))
 
 
 def lvsa_get_device_status(clear: bool = False) -> int:

@@ -27,9 +27,11 @@
 #include <cudaTypedefs.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <mutex>
+#include <vector>
 
 #include "lvsa.h"
 #include "sm100.cuh"
@@ -79,7 +81,8 @@ struct KernelParams {
   CUtensorMap tm_v;
   __nv_bfloat16* out;
   const int32_t* lists;
-  int T, P, H, L;
+  int T, P, H, L;    // H: heads in this launch (grid.y)
+  int HS;            // heads per token row in memory (H for a whole tensor, more for a band of heads)
   int straddle;      // 1: CTA c takes query rows [256c, 256c+256) of the whole frame-major sequence
   int qblocks;       // straddle == 0: ceil(P / 256) CTAs per query frame
   int nblocks;       // CTAs per (batch, head)
@@ -596,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
           tc_fence_after();
           const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a frame with no valid list entry: zero output
           const bool valid = row < r1;
-          __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * ltok + row) * p.H + h) * D;
+          __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * ltok + row) * p.HS + h) * D;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
@@ -668,14 +671,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [batch][tokens][heads*d] bf16 viewed as a 3-D tensor {heads*d, tokens, batch};
+// A band of H heads out of rows of HS heads: [batch][tokens][HS*d] bf16 starting at `base`
+// (the band's first head) viewed as a 3-D tensor {H*d, tokens, batch} with row pitch HS*d;
 // one box = 64 columns (128 bytes, one swizzle row) x 128 tokens.
-bool make_map(CUtensorMap* tm, const void* base, int B, long long tokens, int H, int d) {
+bool make_map(CUtensorMap* tm, const void* base, int B, long long tokens, int H, int HS, int d) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(H) * d, static_cast<cuuint64_t>(tokens),
                         static_cast<cuuint64_t>(B)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(H) * d * 2, static_cast<cuuint64_t>(tokens) * H * d * 2};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(HS) * d * 2, static_cast<cuuint64_t>(tokens) * HS * d * 2};
   cuuint32_t box[3] = {64, kBM, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -711,22 +715,32 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 }  // namespace
 }  // namespace lvsa
 
-// ------------------------------------------------------------------ C ABI
-extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* v, const int32_t* lists, int L,
-                                      int T, int tokens_per_frame, int heads, int d, int batch, float scale,
-                                      void* out, void* stream) {
-  using namespace lvsa;
-  const int P = tokens_per_frame;
-  if (!q || !k || !v || !lists || !out) return LVSA_ERR_INVALID_ARG;
+namespace lvsa {
+namespace {
+
+// Checks shared by both attention entry points (no CUDA call).
+lvsa_status check_sizes(int L, int T, int P, int heads, int d, int batch, float scale) {
   if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T) return LVSA_ERR_INVALID_ARG;
   if (heads > 65535 || batch > 65535) return LVSA_ERR_INVALID_ARG;
   if (static_cast<long long>(T) * P > INT_MAX) return LVSA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return LVSA_ERR_INVALID_ARG;
-  if (out == q || out == k || out == v) return LVSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lists) & 3u))
-    return LVSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return LVSA_ERR_UNSUPPORTED;
   if (T > kMaxT) return LVSA_ERR_UNSUPPORTED;
+  return LVSA_OK;
+}
+
+lvsa_status check_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) return LVSA_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess) return LVSA_ERR_CUDA;
+  return major == 10 ? LVSA_OK : LVSA_ERR_UNSUPPORTED;
+}
+
+// One launch over `heads` heads whose rows hold `head_stride` heads; q, k, v, out point
+// at the band's first head.  Arguments are already validated.
+lvsa_status launch_band(const void* q, const void* k, const void* v, const int32_t* lists, int L, int T, int P,
+                        int heads, int head_stride, int d, int batch, float scale, void* out, cudaStream_t st,
+                        int dev) {
   const int qblocks = (P + kQTiles * kBM - 1) / (kQTiles * kBM);
   // frames of at least 256 tokens: query blocks of 256 rows run over the whole
   // sequence (a block may hold the end of one frame and the start of the next);
@@ -735,23 +749,18 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   const long long nblocks = straddle ? (static_cast<long long>(T) * P + kQTiles * kBM - 1) / (kQTiles * kBM)
                                      : static_cast<long long>(T) * qblocks;
   if (nblocks > INT_MAX) return LVSA_ERR_INVALID_ARG;
-
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LVSA_ERR_CUDA;
-  int major = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return LVSA_ERR_CUDA;
-  if (major != 10) return LVSA_ERR_UNSUPPORTED;
-
   KernelParams kp;
   const long long tokens = static_cast<long long>(T) * P;
-  if (!make_map(&kp.tm_q, q, batch, tokens, heads, d) || !make_map(&kp.tm_k, k, batch, tokens, heads, d) ||
-      !make_map(&kp.tm_v, v, batch, tokens, heads, d))
+  if (!make_map(&kp.tm_q, q, batch, tokens, heads, head_stride, d) ||
+      !make_map(&kp.tm_k, k, batch, tokens, heads, head_stride, d) ||
+      !make_map(&kp.tm_v, v, batch, tokens, heads, head_stride, d))
     return LVSA_ERR_CUDA;
   kp.out = static_cast<__nv_bfloat16*>(out);
   kp.lists = lists;
   kp.T = T;
   kp.P = P;
   kp.H = heads;
+  kp.HS = head_stride;
   kp.L = L;
   kp.qblocks = qblocks;
   kp.straddle = straddle;
@@ -759,8 +768,130 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   kp.scale_log2 = sc * 1.4426950408889634f;
   kp.wait_cycles = static_cast<long long>(static_cast<double>(g_wait_ns) * kBudgetCyclesPerNs);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch<128>(kp, batch, st, dev) : launch<64>(kp, batch, st, dev);
+}
+
+// Streams and events of the host-buffer path, created once per device and kept.
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  std::vector<cudaEvent_t> ev;  // 2 per band + 2
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+
+lvsa_status pipe_for(int dev, int bands, HostPipe** out) {
+  if (dev < 0 || dev >= 64) return LVSA_ERR_UNSUPPORTED;
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.h2d && cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess) return LVSA_ERR_CUDA;
+  if (!hp.d2h && cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess) return LVSA_ERR_CUDA;
+  const size_t need = 2 * static_cast<size_t>(bands) + 2;
+  while (hp.ev.size() < need) {
+    cudaEvent_t e;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return LVSA_ERR_CUDA;
+    hp.ev.push_back(e);
+  }
+  *out = &hp;
+  return LVSA_OK;
+}
+
+bool disjoint(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x + bytes <= y || y + bytes <= x;
+}
+
+}  // namespace
+}  // namespace lvsa
+
+// ------------------------------------------------------------------ C ABI
+extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* v, const int32_t* lists, int L,
+                                      int T, int tokens_per_frame, int heads, int d, int batch, float scale,
+                                      void* out, void* stream) {
+  using namespace lvsa;
+  const int P = tokens_per_frame;
+  if (!q || !k || !v || !lists || !out) return LVSA_ERR_INVALID_ARG;
+  if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T) return LVSA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return LVSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lists) & 3u))
+    return LVSA_ERR_INVALID_ARG;
+  const lvsa_status cs = check_sizes(L, T, P, heads, d, batch, scale);
+  if (cs != LVSA_OK) return cs;
+  int dev = 0;
+  const lvsa_status ds = check_device(&dev);
+  if (ds != LVSA_OK) return ds;
+  return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale, out, static_cast<cudaStream_t>(stream),
+                     dev);
+}
+
+extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_host, const void* v_host,
+                                           const int32_t* lists_host, int L, int T, int tokens_per_frame, int heads,
+                                           int d, int batch, float scale, void* out_host, void* q_dev, void* k_dev,
+                                           void* v_dev, int32_t* lists_dev, void* out_dev, int heads_per_band,
+                                           void* stream) {
+  using namespace lvsa;
+  const int P = tokens_per_frame;
+  if (!q_host || !k_host || !v_host || !lists_host || !out_host) return LVSA_ERR_INVALID_ARG;
+  if (!q_dev || !k_dev || !v_dev || !lists_dev || !out_dev) return LVSA_ERR_INVALID_ARG;
+  if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T) return LVSA_ERR_INVALID_ARG;
+  if (heads_per_band < 0 || heads_per_band > heads) return LVSA_ERR_INVALID_ARG;
+  if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(v_dev) || !aligned16(out_dev) ||
+      (reinterpret_cast<uintptr_t>(lists_dev) & 3u))
+    return LVSA_ERR_INVALID_ARG;
+  const lvsa_status cs = check_sizes(L, T, P, heads, d, batch, scale);
+  if (cs != LVSA_OK) return cs;
+  const size_t row_bytes = static_cast<size_t>(heads) * d * 2;
+  const size_t rows = static_cast<size_t>(batch) * T * P;
+  const size_t bytes = rows * row_bytes;
+  if (!disjoint(out_dev, q_dev, bytes) || !disjoint(out_dev, k_dev, bytes) || !disjoint(out_dev, v_dev, bytes))
+    return LVSA_ERR_INVALID_ARG;
+  if (!disjoint(out_host, q_host, bytes) || !disjoint(out_host, k_host, bytes) || !disjoint(out_host, v_host, bytes))
+    return LVSA_ERR_INVALID_ARG;
+  int dev = 0;
+  const lvsa_status ds = check_device(&dev);
+  if (ds != LVSA_OK) return ds;
+  // default: one head per band, so that only one head's upload (before the first kernel) and one
+  // head's readback (after the last) are not hidden; a band of one head still fills the GPU at
+  // video sizes (T*P/256 query blocks per batch entry)
+  const int hb = heads_per_band > 0 ? heads_per_band : 1;
+  const int bands = (heads + hb - 1) / hb;
+  std::lock_guard<std::mutex> g(g_pipe_mu);
+  HostPipe* hp = nullptr;
+  lvsa_status r = pipe_for(dev, bands, &hp);
+  if (r != LVSA_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev_start = hp->ev[2 * bands], ev_done = hp->ev[2 * bands + 1];
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // the copies into the staging buffers wait for earlier work on the caller's stream
+  if (!ok(cudaEventRecord(ev_start, st)) || !ok(cudaStreamWaitEvent(hp->h2d, ev_start, 0)) ||
+      !ok(cudaStreamWaitEvent(hp->d2h, ev_start, 0)))
+    return LVSA_ERR_CUDA;
+  if (!ok(cudaMemcpyAsync(lists_dev, lists_host, static_cast<size_t>(T) * L * 4, cudaMemcpyHostToDevice, hp->h2d)))
+    return LVSA_ERR_CUDA;
+  const char* src[3] = {static_cast<const char*>(q_host), static_cast<const char*>(k_host),
+                        static_cast<const char*>(v_host)};
+  char* dst[3] = {static_cast<char*>(q_dev), static_cast<char*>(k_dev), static_cast<char*>(v_dev)};
+  for (int gi = 0; gi < bands; ++gi) {
+    const int h0 = gi * hb;
+    const int hn = std::min(hb, heads - h0);
+    const size_t off = static_cast<size_t>(h0) * d * 2;
+    const size_t width = static_cast<size_t>(hn) * d * 2;
+    cudaEvent_t ev_in = hp->ev[2 * gi], ev_k = hp->ev[2 * gi + 1];
+    // band gi of Q, K, V: a column band of every token row
+    for (int t = 0; t < 3; ++t)
+      if (!ok(cudaMemcpy2DAsync(dst[t] + off, row_bytes, src[t] + off, row_bytes, width, rows, cudaMemcpyHostToDevice,
+                                hp->h2d)))
+        return LVSA_ERR_CUDA;
+    if (!ok(cudaEventRecord(ev_in, hp->h2d)) || !ok(cudaStreamWaitEvent(st, ev_in, 0))) return LVSA_ERR_CUDA;
+    r = launch_band(dst[0] + off, dst[1] + off, dst[2] + off, lists_dev, L, T, P, hn, heads, d, batch, scale,
+                    static_cast<char*>(out_dev) + off, st, dev);
+    if (r != LVSA_OK) return r;
+    if (!ok(cudaEventRecord(ev_k, st)) || !ok(cudaStreamWaitEvent(hp->d2h, ev_k, 0))) return LVSA_ERR_CUDA;
+    if (!ok(cudaMemcpy2DAsync(static_cast<char*>(out_host) + off, row_bytes, static_cast<const char*>(out_dev) + off,
+                              row_bytes, width, rows, cudaMemcpyDeviceToHost, hp->d2h)))
+      return LVSA_ERR_CUDA;
+  }
+  // later work on the caller's stream sees the whole output in host memory
+  if (!ok(cudaEventRecord(ev_done, hp->d2h)) || !ok(cudaStreamWaitEvent(st, ev_done, 0))) return LVSA_ERR_CUDA;
+  return LVSA_OK;
 }
 
 extern "C" lvsa_status lvsa_get_device_status(unsigned int* flags, int clear) {

@@ -18,8 +18,8 @@
  *    no output has been written and nothing was launched.
  *  - The library never allocates device memory and never frees caller memory:
  *    the caller owns every buffer it passes.
- *  - Thread safety: lvsa_build_frame_lists is pure; lvsa_attention may be called
- *    from several host threads on different streams.
+ *  - Thread safety: lvsa_build_frame_lists is pure; lvsa_attention and
+ *    lvsa_attention_host may be called from several host threads.
  */
 #ifndef LVSA_H
 #define LVSA_H
@@ -122,6 +122,46 @@ lvsa_status lvsa_attention(const void* q, const void* k, const void* v,
                            const int32_t* lists, int L, int T, int tokens_per_frame,
                            int heads, int d, int batch, float scale,
                            void* out, void* stream);
+
+/*
+ * lvsa_attention_host -- lvsa_attention on HOST inputs and output, with the
+ * transfers pipelined against the kernel by bands of heads.
+ *
+ * Defines the same output as lvsa_attention.  Heads are independent in the
+ * method (the frame lists A(t) are indexed by query frame and step only, and
+ * shared by every head and batch entry: gist.science summary, section 2
+ * "Core Mechanism"), so the call is cut into bands of heads: band g's Q, K, V
+ * columns are copied host -> device, its attention kernel runs, and its output
+ * columns are copied device -> host; the upload of band g+1 and the readback
+ * of band g-1 overlap the kernel of band g.
+ *
+ * Arguments:
+ *   q_host, k_host, v_host  HOST bf16 [batch][T*tokens_per_frame][heads][d].
+ *            Page-locked (pinned) memory is needed for the copies to overlap.
+ *   lists_host  HOST int32 [T][L] (as written by lvsa_build_frame_lists).
+ *   L, T, tokens_per_frame, heads, d, batch, scale  as lvsa_attention.
+ *   out_host HOST bf16, same layout as q_host; must not overlap q/k/v_host.
+ *   q_dev, k_dev, v_dev, out_dev  DEVICE staging buffers of the full tensor
+ *            size (batch*T*tokens_per_frame*heads*d bf16 each), caller-owned,
+ *            16-byte aligned; out_dev must not overlap q/k/v_dev.  On return
+ *            from the stream they hold the inputs and the output.
+ *   lists_dev   DEVICE int32 [T][L] staging buffer, 4-byte aligned.
+ *   heads_per_band  heads per band, 1..heads; 0 = one head per band.
+ *   stream   a cudaStream_t (as void*), NULL = default stream.  The copies
+ *            start after the work already queued on `stream`; work queued on
+ *            `stream` after this call runs after out_host is written.  The
+ *            library keeps two internal copy streams and a set of events per
+ *            device (created on first use, never freed); calls are serialised
+ *            by a lock while they are queued.
+ * Behaviour: asynchronous; errors as lvsa_attention (a failure part-way
+ * returns LVSA_ERR_CUDA and leaves out_host partly written).  Synchronise
+ * `stream` before reading out_host.
+ */
+lvsa_status lvsa_attention_host(const void* q_host, const void* k_host, const void* v_host,
+                                const int32_t* lists_host, int L, int T, int tokens_per_frame,
+                                int heads, int d, int batch, float scale, void* out_host,
+                                void* q_dev, void* k_dev, void* v_dev, int32_t* lists_dev,
+                                void* out_dev, int heads_per_band, void* stream);
 
 /*
  * lvsa_get_device_status -- device status bits (LVSA_DEV_*) of the current

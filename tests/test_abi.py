@@ -71,3 +71,35 @@ def test_attention_argument_validation_without_gpu(lib):
 
     if not cuda_available():
         assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
+
+
+def test_host_path_argument_validation_without_gpu(lib):
+    A = 1 << 20       # 16-byte aligned fake addresses; validation fails before any is used
+    n = 8 * 64 * 2 * 64 * 2   # bytes of one [1, 8*64, 2, 64] bf16 tensor
+    good = [A, A + n, A + 2 * n, A + 3 * n, 4, 8, 64, 2, 64, 1, 0.0, A + 4 * n,
+            A + 8 * n, A + 9 * n, A + 10 * n, A + 11 * n, A + 12 * n, 0, 0]
+    names = ["q_host", "k_host", "v_host", "lists_host", "L", "T", "P", "H", "d", "B", "scale", "out_host",
+             "q_dev", "k_dev", "v_dev", "lists_dev", "out_dev", "heads_per_band", "stream"]
+
+    def call(**kw):
+        a = list(good)
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return lib.lvsa_attention_host_raw(*a)
+
+    INV = lib.LVSA_ERR_INVALID_ARG
+    for ptr in ("q_host", "k_host", "v_host", "lists_host", "out_host", "q_dev", "k_dev", "v_dev", "lists_dev",
+                "out_dev"):
+        assert call(**{ptr: 0}) == INV, ptr
+    assert call(heads_per_band=-1) == INV
+    assert call(heads_per_band=3) == INV          # more than the 2 heads
+    assert call(q_dev=A + 8 * n + 8) == INV       # device staging not 16-byte aligned
+    assert call(lists_dev=A + 11 * n + 2) == INV  # int32 misaligned
+    assert call(out_dev=A + 8 * n + 64) == INV    # output staging overlaps q_dev
+    assert call(out_host=A + n // 2) == INV       # host output overlaps q_host
+    assert call(L=0) == INV and call(T=0) == INV
+    assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
+    from conftest import cuda_available
+
+    if not cuda_available():
+        assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)

@@ -233,3 +233,41 @@ def test_frame_without_valid_entries_gives_zeros(gpu_lib):
     rows = [r for r in range(T * P) if r // P != 4]
     ref = OA.sparse_attention_rows(q, k, v, good, P, rows)
     assert_close(out[:, rows], ref, "other frames")
+
+
+def run_host_path(lib, q, k, v, lists_np, P, heads_per_band=0, scale=0.0):
+    """The host-buffer entry point: CPU tensors in, CPU tensor out, staging buffers on the GPU."""
+    qh, kh, vh = (x.cpu().contiguous().pin_memory() for x in (q, k, v))
+    lh = torch.from_numpy(np.ascontiguousarray(lists_np, dtype=np.int32))
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd, od = (torch.empty(qh.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    ld = torch.empty(lh.shape, dtype=torch.int32, device="cuda")
+    lib.lvsa_attention_host(qh, kh, vh, lh, P, oh, qd, kd, vd, ld, od, scale=scale, heads_per_band=heads_per_band)
+    torch.cuda.synchronize()
+    return oh
+
+
+@pytest.mark.parametrize("T,P,H,d,B,C,W,s,hb", [
+    (8, 64, 2, 64, 1, 4, 2, 1, 1),      # tiny shape, one head per band
+    (8, 64, 2, 64, 1, 4, 2, 1, 0),      # automatic bands
+    (6, 300, 3, 128, 2, 3, 1, 4, 2),    # straddling query blocks, batch 2, uneven bands (2 + 1 heads)
+    (5, 96, 5, 64, 1, 5, 2, 0, 3),      # dense lists, ragged frames, bands of 3 + 2
+])
+def test_host_buffer_path_equals_device_path(gpu_lib, T, P, H, d, B, C, W, s, hb):
+    q, k, v = make(T, P, H, d, B=B, seed=11)
+    lists = gpu_lib.lvsa_build_frame_lists(T, C, W, s)
+    dev_out = run_kernel(gpu_lib, q, k, v, lists, P).cpu()
+    host_out = run_host_path(gpu_lib, q, k, v, lists, P, heads_per_band=hb)
+    # same kernel on the same bf16 inputs, one band of heads at a time: identical bits
+    assert torch.equal(host_out.view(torch.int16), dev_out.view(torch.int16))
+    ref = OA.sparse_attention(q.cpu(), k.cpu(), v.cpu(), OL.frame_lists(T, C, W, s), P)
+    assert_close(host_out.float().numpy(), ref, "host-buffer path")
+
+
+def test_host_buffer_path_full_size_heads(gpu_lib):
+    """Wan-1.3B 1x shape (T=21, P=1560, 12 heads): automatic bands, bit-identical to the device path."""
+    q, k, v = make(21, 1560, 12, 128, seed=5)
+    lists = gpu_lib.lvsa_build_frame_lists(21, 21, 9, 0)
+    dev_out = run_kernel(gpu_lib, q, k, v, lists, 1560).cpu()
+    host_out = run_host_path(gpu_lib, q, k, v, lists, 1560)
+    assert torch.equal(host_out.view(torch.int16), dev_out.view(torch.int16))
