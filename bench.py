@@ -373,6 +373,9 @@ def run_lvsa(args, rank, world, local):
                      "peak_source": f"{peak_src} bf16 dense (burst)",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                      "kernel_ms_avg": kern_avg_ms, "flops_per_launch": F},
+        "kernel_ms_over_steps": {"steps": f"s = {args.warmup}..{args.warmup + args.steps - 1}",
+                                 "mean": kern_avg_ms, "median": statistics.median(kernel_ms),
+                                 "min": min(kernel_ms), "max": max(kernel_ms)},
         "e2e": {"value": F / (e2e_ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "call": "lvsa_attention_host (pinned host buffers; copies pipelined by bands of "
