@@ -514,13 +514,9 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         }
         tc_fence_after();
         pv(0, v_addr, n_cur, j > 0, 0, 4);
-        if (!wait_all(bar_p + 0, j & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        pv(0, v_addr, n_cur, j > 0, 4, 8);
-        commit(bar_o + 0);
+        // the next K tile is waited for while the softmax finishes P_0(j), so that nothing but the
+        // P_0 hand-off stands between PV_0(j) and QK_0(j+1); commits that nobody waits on soon go
+        // after the next group of MMAs
         int ki = -1;
         uint32_t k_addr = 0;
         if (has_next) {
@@ -530,10 +526,18 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
             ok = false;
             break;
           }
-          tc_fence_after();
+        }
+        if (!wait_all(bar_p + 0, j & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        pv(0, v_addr, n_cur, j > 0, 4, 8);
+        if (has_next) {
           qk(0, k_addr, n_next);
           commit(bar_s + 0);
         }
+        commit(bar_o + 0);
         if (has1) {
           if (!wait_all(bar_ph + 1, j & 1)) {
             ok = false;
@@ -547,14 +551,14 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
           }
           tc_fence_after();
           pv(1, v_addr, n_cur, j > 0, 4, 8);
+          if (has_next) {
+            qk(1, k_addr, n_next);
+            commit(bar_s + 1);
+          }
           commit(bar_o + 1);
         }
         commit(bar_empty + slot_of(vi));
         if (!has_next) break;
-        if (has1) {
-          qk(1, k_addr, n_next);
-          commit(bar_s + 1);
-        }
         commit(bar_empty + slot_of(ki));
         n_cur = n_next;
       }
