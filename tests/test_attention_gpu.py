@@ -285,3 +285,18 @@ def test_host_buffer_path_full_size_heads(gpu_lib):
     dev_out = run_kernel(gpu_lib, q, k, v, lists, 1560).cpu()
     host_out = run_host_path(gpu_lib, q, k, v, lists, 1560)
     assert torch.equal(host_out.view(torch.int16), dev_out.view(torch.int16))
+
+
+def test_host_buffer_path_pageable_memory(gpu_lib):
+    """Pageable (not pinned) host tensors: the copies stall instead of overlapping, the result is the same."""
+    T, P, H, d = 6, 200, 3, 64
+    q, k, v = make(T, P, H, d, seed=21)
+    lists = gpu_lib.lvsa_build_frame_lists(T, 4, 2, 2)
+    dev_out = run_kernel(gpu_lib, q, k, v, lists, P).cpu()
+    qh, kh, vh = (x.cpu().contiguous() for x in (q, k, v))
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16)
+    qd, kd, vd, od = (torch.empty(qh.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    ld = torch.empty(lists.shape, dtype=torch.int32, device="cuda")
+    gpu_lib.lvsa_attention_host(qh, kh, vh, torch.from_numpy(lists), P, oh, qd, kd, vd, ld, od)
+    torch.cuda.synchronize()
+    assert torch.equal(oh.view(torch.int16), dev_out.view(torch.int16))
