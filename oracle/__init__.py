@@ -28,7 +28,7 @@ Diffusion"):
     count is the same at every step; a few frames may be an anchor one extra
     time when T is not a multiple of the stride.
 
-Readings where the pages are silent or disagree (each is listed in the design doc):
+Readings where the pages are silent or disagree:
   * rotation offset is ``step mod T`` (section 三 of the techwalker article);
   * anchors sit at the fractional stride floor(k*T/G), k = 0..G-1, so there
     are always G distinct anchors;
