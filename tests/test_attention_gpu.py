@@ -300,3 +300,20 @@ def test_host_buffer_path_pageable_memory(gpu_lib):
     gpu_lib.lvsa_attention_host(qh, kh, vh, torch.from_numpy(lists), P, oh, qd, kd, vd, ld, od)
     torch.cuda.synchronize()
     assert torch.equal(oh.view(torch.int16), dev_out.view(torch.int16))
+
+
+@pytest.mark.parametrize("P,d", [(16, 64), (40, 128)])
+def test_maximum_frame_count(gpu_lib, P, d):
+    """T = 4096, the largest frame count the kernel's frame bitmaps cover: sampled rows against the oracle,
+    including the first and last frames (anchors wrap around the end of the sequence)."""
+    T, C, W, s = 4096, 7, 3, 4093
+    q, k, v = make(T, P, 1, d, seed=31)
+    lists = gpu_lib.lvsa_build_frame_lists(T, C, W, s)
+    out = run_kernel(gpu_lib, q, k, v, lists, P)
+    g = np.random.default_rng(5)
+    frames = sorted(set([0, 1, 2047, 4094, 4095] + list(g.choice(T, 5, replace=False))))
+    rows = [f * P + r for f in frames for r in range(P)]
+    got = out[:, rows].float().cpu().numpy()
+    ref = OA.sparse_attention_rows(q.cpu(), k.cpu(), v.cpu(), OL.frame_lists(T, C, W, s), P, rows)
+    assert_close(got, ref, f"T=4096 P={P} d={d}")
+    assert torch.isfinite(out).all()
