@@ -775,9 +775,11 @@ lvsa_status launch_band(const void* q, const void* k, const void* v, const int32
   return d == 128 ? launch<128>(kp, batch, st, dev) : launch<64>(kp, batch, st, dev);
 }
 
-// Streams and events of the host-buffer path, created once per device and kept.
+// Streams and events of the host-buffer path, created once per device and kept: one upload and one
+// readback stream, and two streams the band kernels alternate on, so that a band's CTAs start on the
+// SMs the previous band's last wave leaves free.
 struct HostPipe {
-  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaStream_t h2d = nullptr, d2h = nullptr, k[2] = {nullptr, nullptr};
   std::vector<cudaEvent_t> ev;  // 2 per band + 2
 };
 std::mutex g_pipe_mu;
@@ -788,6 +790,8 @@ lvsa_status pipe_for(int dev, int bands, HostPipe** out) {
   HostPipe& hp = g_pipe[dev];
   if (!hp.h2d && cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess) return LVSA_ERR_CUDA;
   if (!hp.d2h && cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess) return LVSA_ERR_CUDA;
+  for (int i = 0; i < 2; ++i)
+    if (!hp.k[i] && cudaStreamCreateWithFlags(&hp.k[i], cudaStreamNonBlocking) != cudaSuccess) return LVSA_ERR_CUDA;
   const size_t need = 2 * static_cast<size_t>(bands) + 2;
   while (hp.ev.size() < need) {
     cudaEvent_t e;
@@ -884,16 +888,18 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
       if (!ok(cudaMemcpy2DAsync(dst[t] + off, row_bytes, src[t] + off, row_bytes, width, rows, cudaMemcpyHostToDevice,
                                 hp->h2d)))
         return LVSA_ERR_CUDA;
-    if (!ok(cudaEventRecord(ev_in, hp->h2d)) || !ok(cudaStreamWaitEvent(st, ev_in, 0))) return LVSA_ERR_CUDA;
+    cudaStream_t ks = hp->k[gi & 1];
+    if (!ok(cudaEventRecord(ev_in, hp->h2d)) || !ok(cudaStreamWaitEvent(ks, ev_in, 0))) return LVSA_ERR_CUDA;
     r = launch_band(dst[0] + off, dst[1] + off, dst[2] + off, lists_dev, L, T, P, hn, heads, d, batch, scale,
-                    static_cast<char*>(out_dev) + off, st, dev);
+                    static_cast<char*>(out_dev) + off, ks, dev);
     if (r != LVSA_OK) return r;
-    if (!ok(cudaEventRecord(ev_k, st)) || !ok(cudaStreamWaitEvent(hp->d2h, ev_k, 0))) return LVSA_ERR_CUDA;
+    if (!ok(cudaEventRecord(ev_k, ks)) || !ok(cudaStreamWaitEvent(hp->d2h, ev_k, 0))) return LVSA_ERR_CUDA;
     if (!ok(cudaMemcpy2DAsync(static_cast<char*>(out_host) + off, row_bytes, static_cast<const char*>(out_dev) + off,
                               row_bytes, width, rows, cudaMemcpyDeviceToHost, hp->d2h)))
       return LVSA_ERR_CUDA;
   }
-  // later work on the caller's stream sees the whole output in host memory
+  // later work on the caller's stream sees the whole output in host memory (every band's readback
+  // waited for its kernel, so this also orders every kernel before that work)
   if (!ok(cudaEventRecord(ev_done, hp->d2h)) || !ok(cudaStreamWaitEvent(st, ev_done, 0))) return LVSA_ERR_CUDA;
   return LVSA_OK;
 }

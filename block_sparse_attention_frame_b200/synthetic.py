@@ -66,6 +66,9 @@ WORKLOADS = {
     "wan14b_6x": Workload("wan14b_6x", T=121, P=1560, H=40, d=128, C=21, W=9, seed=1004),
     # HunyuanVideo-1.5 at 1.5x horizon (193 video frames = 49 latent frames)
     "hunyuan1.5_1.5x": Workload("hunyuan1.5_1.5x", T=49, P=1560, H=16, d=128, C=33, W=13, seed=1005),
+    # HunyuanVideo-1.5 at 2x horizon (257 video frames = 65 latent frames; the pages' out-of-memory case for
+    # dense attention in the full model on an 80 GB GPU)
+    "hunyuan1.5_2x": Workload("hunyuan1.5_2x", T=65, P=1560, H=16, d=128, C=33, W=13, seed=1006),
     # profiling slice: the Wan-1.3B 6x call with 2 of its 12 heads (Q+K+V+O = 387 MB, still > L2)
     "wan1.3b_6x_h2": Workload("wan1.3b_6x_h2", T=121, P=1560, H=2, d=128, C=21, W=9, seed=1003),
 }

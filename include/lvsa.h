@@ -150,9 +150,10 @@ lvsa_status lvsa_attention(const void* q, const void* k, const void* v,
  *   stream   a cudaStream_t (as void*), NULL = default stream.  The copies
  *            start after the work already queued on `stream`; work queued on
  *            `stream` after this call runs after out_host is written.  The
- *            library keeps two internal copy streams and a set of events per
- *            device (created on first use, never freed); calls are serialised
- *            by a lock while they are queued.
+ *            library keeps four internal streams (upload, readback, and two
+ *            that the band kernels alternate on) and a set of events per device
+ *            (created on first use, never freed); calls are serialised by a
+ *            lock while they are queued.
  * Behaviour: asynchronous; errors as lvsa_attention (a failure part-way
  * returns LVSA_ERR_CUDA and leaves out_host partly written).  Synchronise
  * `stream` before reading out_host.

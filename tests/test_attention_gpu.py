@@ -177,6 +177,7 @@ def sample_rows(T, P, seed, per_frame=40):
     ("wan1.3b_1x", [0]),
     ("wan1.3b_6x", [0, 17, 49]),
     ("hunyuan1.5_1.5x", [0, 2, 31]),
+    ("hunyuan1.5_2x", [0, 40]),
     ("wan14b_6x", [5]),
 ])
 def test_full_size_workloads_sampled_rows(gpu_lib, name, steps):
