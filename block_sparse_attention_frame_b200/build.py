@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "liblvsa.so")
 
 SOURCES = ["lists.cpp", "attention.cu"]
-HEADERS = [os.path.join(INCLUDE, "lvsa.h"), os.path.join(CSRC, "sm100.cuh")]
+HEADERS = [os.path.join(INCLUDE, "lvsa.h"), os.path.join(CSRC, "sm100.cuh"), os.path.join(CSRC, "attention_kernel.cuh")]
 
 
 def nvcc_path() -> str:

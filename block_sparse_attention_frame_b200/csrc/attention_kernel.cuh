@@ -1,0 +1,658 @@
+// Device code of the LVSA attention path for B200 (sm_100a): the attention kernel and its helpers.
+//
+// "LVSA: Training-Free Sparse Attention for Long Video Diffusion" (gist.science technical summary,
+// section 2 "Core Mechanism" and "Complexity"): a query token of frame t attends only to the tokens of the
+// frames in A(t); one softmax over all of them; cost O(T * C * P^2 * d).
+//
+// One CTA per (256-row query block, head, batch entry); 384 threads:
+//   warp 8      TMA producer: both 128-row Q tiles once, then K and V tiles of the frames the block
+//               attends into a 5-slot shared-memory ring.  A block may hold the end of frame fa and the
+//               start of fa + 1; it attends the union of their lists, walked as runs of consecutive
+//               frames (one contiguous token range each, cut into 128-token tiles, the last partial).
+//               The gather is done by TMA coordinates: no mask is ever materialised.
+//   warp 9      TMEM allocator and tcgen05.mma issuer (one elected lane):
+//                 S_i = Q_i K_j^T  into query tile i's S columns (SS form)
+//                 O_i += P_i V_j   with P_i read from TMEM (TS form), in two halves of 64 keys
+//               in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the tensor core works on one
+//               query tile while the other tile's softmax runs.
+//   warps 0-3   softmax of query tile 0, warps 4-7 of query tile 1, one thread per row (TMEM lane):
+//               online softmax in the exp2 domain with a lazily updated running max (O in TMEM is
+//               rescaled only when the max grows by more than 2^8), P written back over the S columns
+//               as bf16; rows of the other frame skip the tiles their frame does not attend.
+//               Epilogue O / l -> bf16 -> HBM.
+// Every wait is bounded: when its time budget runs out the CTA stops, sets a device status bit, lets its
+// in-flight copies and MMAs finish and frees TMEM.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <cmath>
+
+#include "lvsa.h"
+#include "sm100.cuh"
+
+__device__ unsigned int g_lvsa_dev_status = 0;
+
+namespace lvsa {
+using namespace sm100;
+
+constexpr int kBM = 128;          // query rows per tile = MMA M
+constexpr int kBN = 128;          // keys per K/V tile = largest MMA N of QK^T
+constexpr int kQTiles = 2;        // query tiles per CTA, sharing every K/V tile
+constexpr int kThreads = 384;     // warps 0-3: softmax tile 0, 4-7: softmax tile 1, 8: TMA, 9: MMA, 10-11 idle
+// Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup drops to 88 and the
+// two softmax warpgroups rise to 208: 2 x 128 x 208 + 128 x 88 = 64512.
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsControl = 88;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
+constexpr int kTmemCols = 512;    // S/P of tile i: columns [128 i, 128 i + 128); O of tile i: [256 + 128 i, ...)
+constexpr int kOCol0 = 256;
+constexpr int kChunkBytes = kBM * 128;    // one 128-byte-wide swizzle column of a 128-row tile
+constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the max grows by > 2^8
+constexpr int kPolyEvery = 0;             // every kPolyEvery-th element pair takes the FMA-pipe exp2 (0: none)
+
+constexpr int kMaxT = 4096;               // latent frames supported (frame bitmaps in shared memory)
+constexpr int kMapWords = kMaxT / 32;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kTileBytes = kBM * D * 2;
+  static constexpr int kSlots = (D == 128) ? 5 : 10;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = kQTiles * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kSlots * kTileBytes;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kOffMap = kOffBar + kBarBytes;             // two frame bitmaps of kMapWords words
+  static constexpr int kSmemBytes = kOffMap + 2 * kMapWords * 4 + 1024;  // + alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(8 * (1 + 2 * kSlots + 9) + 8 <= kBarBytes, "barrier area");
+};
+
+struct KernelParams {
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  __nv_bfloat16* out;
+  const int32_t* lists;
+  int T, P, H, L;    // H: heads in this launch (grid.y)
+  int HS;            // heads per token row in memory (H for a whole tensor, more for a band of heads)
+  int straddle;      // 1: CTA c takes query rows [256c, 256c+256) of the whole frame-major sequence
+  int qblocks;       // straddle == 0: ceil(P / 256) CTAs per query frame
+  int nblocks;       // CTAs per (batch, head)
+  float scale_log2;  // softmax scale * log2(e)
+  long long wait_cycles;
+};
+
+// ------------------------------------------------------------------ bounded waits
+// The budget is counted in SM clock cycles (a ns budget converted at 2 GHz, so at
+// lower clocks it lasts longer in wall time).  The cycle counter and the abort
+// flag are only looked at every 64 polls: the poll itself must stay cheap, since
+// a slow poll delays the hand-off it waits for.
+constexpr double kBudgetCyclesPerNs = 2.0;
+
+struct Watch {
+  long long budget_cycles;
+  volatile int* abort_flag;  // shared memory, CTA-wide
+};
+
+// Returns false when the budget ran out (status bit set) or another role of the
+// CTA already gave up.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Watch& w) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*w.abort_flag) return false;
+      if (clock64() - t0 > w.budget_cycles) {
+        *w.abort_flag = 1;
+        atomicOr(&g_lvsa_dev_status, LVSA_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Used only while shutting down after an abort: ignores the abort flag.  Copies and
+// MMAs in flight always complete on their own, so the drain allows at least ~1 s
+// whatever the caller's wait budget: a CTA must not exit while a copy can still land
+// in its shared memory.
+constexpr long long kMinDrainCycles = 2000000000ll;
+
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long long budget_cycles) {
+  budget_cycles = budget_cycles > kMinDrainCycles ? budget_cycles : kMinDrainCycles;
+  const long long t0 = clock64();
+  for (uint32_t it = 0; !mbar_try_wait(bar, parity); ++it) {
+    if ((it & 63u) == 63u && clock64() - t0 > budget_cycles) {
+      atomicOr(&g_lvsa_dev_status, LVSA_DEV_TIMEOUT);
+      return;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ K/V tile walk
+// The CTA's query rows belong to frame fa, or to frames fa and fb = fa + 1.  Their
+// frame lists are held as bitmaps over [0, T) (so list order and duplicates do not
+// matter).  The walk visits the union in ascending frame order as runs of
+// consecutive frames with the same membership (bit 0: attended by fa, bit 1: by
+// fb); a run is one contiguous token range, cut into tiles of at most 128 tokens.
+// Every role of the CTA walks the same sequence.
+struct FrameWalk {
+  const uint32_t* ma;
+  const uint32_t* mb;
+  int T, P, nwords;
+  int f = 0, pos = 0, end = 0, mask = 0;
+
+  __device__ FrameWalk(const uint32_t* a, const uint32_t* b_, int T_, int P_)
+      : ma(a), mb(b_), T(T_), P(P_), nwords((T_ + 31) >> 5) {}
+
+  __device__ __forceinline__ int bits(int g) const {
+    return static_cast<int>(((ma[g >> 5] >> (g & 31)) & 1u) | (((mb[g >> 5] >> (g & 31)) & 1u) << 1));
+  }
+
+  __device__ __forceinline__ bool next(int& tok, int& nvalid, int& tmask) {
+    while (pos >= end) {
+      if (f >= T) return false;
+      int wi = f >> 5;
+      uint32_t word = (ma[wi] | mb[wi]) & (0xffffffffu << (f & 31));
+      while (word == 0) {
+        if (++wi >= nwords) {
+          f = T;
+          return false;
+        }
+        word = ma[wi] | mb[wi];
+      }
+      const int f0 = (wi << 5) + __ffs(word) - 1;
+      if (f0 >= T) {
+        f = T;
+        return false;
+      }
+      const int m0 = bits(f0);
+      int f1 = f0;
+      while (f1 + 1 < T && bits(f1 + 1) == m0) ++f1;
+      pos = f0 * P;
+      end = (f1 + 1) * P;
+      mask = m0;
+      f = f1 + 1;
+    }
+    tok = pos;
+    nvalid = min(kBN, end - pos);
+    tmask = mask;
+    pos += nvalid;
+    return true;
+  }
+};
+
+// ------------------------------------------------------------------ softmax of one S tile
+// Thread = one query row.  Loads the row of S from TMEM, masks columns past the
+// run end, updates the running max lazily (rescaling the row of O in TMEM when
+// needed), writes P = 2^(scale*log2e*s - m) as bf16 over the S columns and
+// returns the row sum of P through `l`.  `skip`: the row's frame does not attend
+// the tile (P = 0, max and sum unchanged).  After the first 64 keys of P are
+// stored it arrives on `bar_half`, so the tensor core can run the first half of
+// PV while this thread computes the second half.
+template <int D>
+__device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int nv, int j, bool skip, float sl2,
+                                             float& m, float& l, uint64_t* bar_o, const Watch& w, uint64_t* bar_half) {
+  float s[kBN];
+  tmem_ld32(s_tmem + 0, s + 0);
+  if (nv > 32) tmem_ld32(s_tmem + 32, s + 32);
+  if (nv > 64) tmem_ld32(s_tmem + 64, s + 64);
+  if (nv > 96) tmem_ld32(s_tmem + 96, s + 96);
+  tmem_wait_ld_regs(s + 0);
+  tmem_wait_ld_regs(s + 32);
+  tmem_wait_ld_regs(s + 64);
+  tmem_wait_ld_regs(s + 96);
+  const bool partial = nv < kBN;
+  if (partial) {
+#pragma unroll
+    for (int i = 0; i < kBN; ++i)
+      if (i >= nv) s[i] = -INFINITY;
+  }
+  // row max: 8 chains of 3-input max
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = s[k];
+#pragma unroll
+  for (int i = 8; i < 120; i += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 8 + k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[120 + k]);
+  // a row whose frame does not attend this tile's frames takes no part in it:
+  // its max stays and its P is 2^-inf = 0
+  const float tile_max =
+      skip ? -INFINITY : fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7])) * sl2;
+
+  float alpha = 1.f;
+  if (tile_max > m + kRescaleLog2) {
+    alpha = ex2(m - tile_max);
+    l *= alpha;
+    m = tile_max;
+  }
+  if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+    // O holds PV(0..j-1): wait for PV(j-1), then rescale this thread's row
+    if (!__all_sync(0xffffffffu, wait_bounded(bar_o, (j - 1) & 1, w))) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      tmem_ld32(o_tmem + 32 * c, o);
+      tmem_wait_ld_regs(o);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] *= alpha;
+      tmem_st32(o_tmem + 32 * c, o);
+    }
+  }
+
+  const float2 scale2 = make_float2(sl2, sl2);
+  const float2 negm2 = skip ? make_float2(-INFINITY, -INFINITY) : make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (c == 0 || nv > 32 * c) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float2 x = ffma2(make_float2(s[32 * c + 2 * i], s[32 * c + 2 * i + 1]), scale2, negm2);
+        float2 e;
+        if (kPolyEvery > 0 && !partial && (i % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+          e = exp2_fma2(x);
+        } else {
+          e.x = ex2(x.x);
+          e.y = ex2(x.y);
+        }
+        acc[i & 3] = fadd2(acc[i & 3], e);
+        pk[i] = pack_bf16x2(e.x, e.y);
+      }
+      tmem_st16(s_tmem + 16 * c, pk);  // P overwrites the first half of the S columns
+    }
+    if (c == 1) {
+      // keys 0..63 of P are in TMEM: the MMA warp may start the first half of PV
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_half);
+    }
+  }
+  const float2 t01 = fadd2(acc[0], acc[1]);
+  const float2 t23 = fadd2(acc[2], acc[3]);
+  const float2 tt = fadd2(t01, t23);
+  l += tt.x + tt.y;
+  return true;
+}
+
+// ------------------------------------------------------------------ the kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __grid_constant__ KernelParams p) {
+  using Cf = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + Cf::kOffQ;
+  uint8_t* sRing = smem + Cf::kOffRing;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kOffBar);
+  uint64_t* bar_q = bars;
+  uint64_t* bar_full = bars + 1;
+  uint64_t* bar_empty = bar_full + Cf::kSlots;
+  uint64_t* bar_s = bar_empty + Cf::kSlots;  // [2] S_i(j) ready in TMEM
+  uint64_t* bar_p = bar_s + 2;               // [2] P_i(j) written to TMEM (128 arrivals)
+  uint64_t* bar_o = bar_p + 2;               // [2] PV_i(j) finished
+  uint64_t* bar_ph = bar_o + 2;              // [2] P_i(j) keys 0..63 written (128 arrivals)
+  uint64_t* bar_drain = bar_ph + 2;          // all MMAs of the CTA finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int ltok = p.T * p.P;
+  // query rows [r0, r1) of the frame-major sequence: one frame fa, or fa and fb = fa + 1
+  int r0, r1;
+  if (p.straddle) {
+    r0 = blockIdx.x * (kQTiles * kBM);
+    r1 = min(r0 + kQTiles * kBM, ltok);
+  } else {
+    const int qb = blockIdx.x % p.qblocks;
+    const int t = blockIdx.x / p.qblocks;
+    r0 = t * p.P + qb * (kQTiles * kBM);
+    r1 = min(r0 + kQTiles * kBM, (t + 1) * p.P);
+  }
+  const int fa = r0 / p.P;
+  const int fb = (r1 - 1) / p.P;
+  const bool has1 = r0 + kBM < r1;  // the second query tile has rows
+  uint32_t* map_a = reinterpret_cast<uint32_t*>(smem + Cf::kOffMap);
+  uint32_t* map_b = map_a + kMapWords;
+  {
+    // frame bitmaps of the lists of fa and fb (map_b stays empty when fb == fa)
+    const int nwords = (p.T + 31) >> 5;
+    for (int i = threadIdx.x; i < nwords; i += kThreads) {
+      map_a[i] = 0u;
+      map_b[i] = 0u;
+    }
+    __syncthreads();
+    bool bad = false;
+    const int32_t* la = p.lists + static_cast<size_t>(fa) * p.L;
+    const int32_t* lb = p.lists + static_cast<size_t>(fb) * p.L;
+    const int nset = (fb != fa) ? 2 * p.L : p.L;
+    for (int i = threadIdx.x; i < nset; i += kThreads) {
+      const int f = (i < p.L) ? __ldg(la + i) : __ldg(lb + (i - p.L));
+      if (f < 0 || f >= p.T) {
+        bad = true;
+        continue;
+      }
+      atomicOr((i < p.L ? map_a : map_b) + (f >> 5), 1u << (f & 31));
+    }
+    if (bad) atomicOr(&g_lvsa_dev_status, LVSA_DEV_BAD_LIST);
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < Cf::kSlots; ++i) {
+      mbar_init(bar_full + i, 1);
+      mbar_init(bar_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_s + i, 1);
+      mbar_init(bar_p + i, 4 * 32);
+      mbar_init(bar_o + i, 1);
+      mbar_init(bar_ph + i, 4 * 32);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watch w{p.wait_cycles, abort_flag};
+
+  if (warp >= 8) {
+  regs_dec<kRegsControl>();
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ TMA producer
+    // The whole warp walks the list (warp-uniform control flow); one elected
+    // lane arms the barriers and issues the copies.
+    const int col0 = h * D;
+    const int qrow = r0;
+    if (elect_one()) {
+      mbar_arrive_expect_tx(bar_q, (has1 ? 2 : 1) * Cf::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < Cf::kChunks; ++c) tma_load_3d(sQ + c * kChunkBytes, &p.tm_q, bar_q, col0 + c * 64, qrow, b);
+      if (has1) {
+#pragma unroll
+        for (int c = 0; c < Cf::kChunks; ++c)
+          tma_load_3d(sQ + Cf::kTileBytes + c * kChunkBytes, &p.tm_q, bar_q, col0 + c * 64, qrow + kBM, b);
+      }
+    }
+    __syncwarp();
+    int issued = 0;
+    bool ok = true;
+    auto load = [&](const CUtensorMap* tm, int tok) {
+      const int slot = issued % Cf::kSlots;
+      const uint32_t phase = (issued / Cf::kSlots) & 1;
+      if (!__all_sync(0xffffffffu, wait_bounded(bar_empty + slot, phase ^ 1, w))) {
+        ok = false;
+        return;
+      }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(bar_full + slot, Cf::kTileBytes);
+        uint8_t* dst = sRing + slot * Cf::kTileBytes;
+#pragma unroll
+        for (int c = 0; c < Cf::kChunks; ++c)
+          tma_load_3d(dst + c * kChunkBytes, tm, bar_full + slot, col0 + c * 64, tok, b);
+      }
+      __syncwarp();
+      ++issued;
+    };
+    // consumption order of the MMA warp: K0, V0, K1, V1, ...
+    FrameWalk walk(map_a, map_b, p.T, p.P);
+    int tok, nv, tmask;
+    while (ok && walk.next(tok, nv, tmask)) {
+      load(&p.tm_k, tok);
+      if (ok) load(&p.tm_v, tok);
+    }
+    if (!ok) {
+      // stopped early: let every copy still in flight land before the CTA exits
+      wait_drain(bar_q, 0, p.wait_cycles);
+      const int first = issued > Cf::kSlots ? issued - Cf::kSlots : 0;
+      for (int i = first; i < issued; ++i) wait_drain(bar_full + i % Cf::kSlots, (i / Cf::kSlots) & 1, p.wait_cycles);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    // Per K/V tile j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while softmax 1 works on S_1(j)
+    // the tensor core runs tile 0's products, and the other way round.  Each PV is issued in two
+    // halves (keys 0..63 as soon as the softmax has stored them, then keys 64..127).  The whole warp
+    // runs the schedule (descriptors stay warp-uniform); one elected lane issues.
+    const uint32_t sq = smem_u32(sQ);
+    const uint32_t sr = smem_u32(sRing);
+    const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+    // descriptor of a K-major Q/K tile at byte address a; + (kk>>2)*16 KB + (kk&3)*32 B per 16-wide k-step
+    const uint64_t kdesc0 = smem_desc_sw128(0, 16, 1024);
+    // descriptor of an MN-major V tile: 64-wide d chunks 16 KB apart (LBO), 8-key groups 1 KB apart (SBO)
+    const uint64_t vdesc0 = smem_desc_sw128(0, kChunkBytes, 1024);
+    auto qk = [&](int i, uint32_t k_addr, int n_mma) {
+      const uint64_t qd = kdesc0 + ((sq + i * Cf::kTileBytes) >> 4);
+      const uint64_t kd = kdesc0 + (k_addr >> 4);
+      const uint32_t idesc = idesc_bf16_f32(kBM, n_mma, false);
+      const bool leader = elect_one();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
+        if (leader) mma_ss(tmem + 128 * i, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate, int k_lo, int k_hi) {
+      const uint64_t vd = vdesc0 + (v_addr >> 4);
+      const bool leader = elect_one();
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        if (kk < k_lo) continue;
+        if (kk >= k_hi || kk * 16 >= n_mma) break;
+        if (leader)
+          mma_ts(tmem + kOCol0 + 128 * i, tmem + 128 * i + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
+                 (accumulate || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) mma_commit(bar);
+      __syncwarp();
+    };
+    auto slot_of = [&](int idx) { return idx % Cf::kSlots; };
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_bounded(bar, parity, w));
+    };
+    auto wait_full = [&](int idx) { return wait_all(bar_full + slot_of(idx), (idx / Cf::kSlots) & 1); };
+
+    int cidx = 0;
+    bool ok = wait_all(bar_q, 0);
+    FrameWalk walk(map_a, map_b, p.T, p.P);
+    int tok, nv, tmask;
+    if (ok && walk.next(tok, nv, tmask)) {
+      int n_cur = (nv + 15) & ~15;
+      const int k0 = cidx++;
+      ok = wait_full(k0);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t k_addr = sr + slot_of(k0) * Cf::kTileBytes;
+        qk(0, k_addr, n_cur);
+        commit(bar_s + 0);
+        if (has1) {
+          qk(1, k_addr, n_cur);
+          commit(bar_s + 1);
+        }
+        commit(bar_empty + slot_of(k0));
+      }
+      for (int j = 0; ok; ++j) {
+        int tok_n, nv_n, tmask_n;
+        const bool has_next = walk.next(tok_n, nv_n, tmask_n);
+        const int n_next = (nv_n + 15) & ~15;
+        const int vi = cidx++;
+        const uint32_t v_addr = sr + slot_of(vi) * Cf::kTileBytes;
+        if (!wait_all(bar_ph + 0, j & 1) || !wait_full(vi)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        pv(0, v_addr, n_cur, j > 0, 0, 4);
+        // the next K tile is waited for while the softmax finishes P_0(j), so that nothing but the
+        // P_0 hand-off stands between PV_0(j) and QK_0(j+1); commits that nobody waits on soon go
+        // after the next group of MMAs
+        int ki = -1;
+        uint32_t k_addr = 0;
+        if (has_next) {
+          ki = cidx++;
+          k_addr = sr + slot_of(ki) * Cf::kTileBytes;
+          if (!wait_full(ki)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!wait_all(bar_p + 0, j & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        pv(0, v_addr, n_cur, j > 0, 4, 8);
+        if (has_next) {
+          qk(0, k_addr, n_next);
+          commit(bar_s + 0);
+        }
+        commit(bar_o + 0);
+        if (has1) {
+          if (!wait_all(bar_ph + 1, j & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv(1, v_addr, n_cur, j > 0, 0, 4);
+          if (!wait_all(bar_p + 1, j & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          pv(1, v_addr, n_cur, j > 0, 4, 8);
+          if (has_next) {
+            qk(1, k_addr, n_next);
+            commit(bar_s + 1);
+          }
+          commit(bar_o + 1);
+        }
+        commit(bar_empty + slot_of(vi));
+        if (!has_next) break;
+        commit(bar_empty + slot_of(ki));
+        n_cur = n_next;
+      }
+    }
+    // every MMA issued must be complete before TMEM is released
+    commit(bar_drain);
+    wait_drain(bar_drain, 0, p.wait_cycles);
+    __syncwarp();
+  }
+  } else {
+    regs_inc<kRegsSoftmax>();
+    // ------------------------------------------------------------ softmax + epilogue (warps 0-7)
+    const int qi = warp >> 2;            // query tile of this warpgroup
+    const int r = threadIdx.x & 127;     // row within the tile = TMEM lane
+    if (qi == 0 || has1) {
+      const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const uint32_t s_tmem = tmem + lane_off + 128 * qi;
+      const uint32_t o_tmem = tmem + lane_off + kOCol0 + 128 * qi;
+      float m = -INFINITY;  // running max of scale*log2(e)*s (possibly stale by < 8)
+      float l = 0.f;        // running sum of 2^(scaled s - m)
+      bool ok = true;
+      int j = 0;
+      const int row = r0 + qi * kBM + r;  // query row in the frame-major sequence
+      const int rbit = (row / p.P == fa) ? 1 : 2;
+      FrameWalk walk(map_a, map_b, p.T, p.P);
+      int tok, nv, tmask;
+      while (walk.next(tok, nv, tmask)) {
+        ok = __all_sync(0xffffffffu, wait_bounded(bar_s + qi, j & 1, w));
+        if (!ok) break;
+        tc_fence_after();
+        ok = softmax_tile<D>(s_tmem, o_tmem, nv, j, (tmask & rbit) == 0, p.scale_log2, m, l, bar_o + qi, w,
+                             bar_ph + qi);
+        if (!ok) break;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_p + qi);
+        ++j;
+      }
+      if (ok && j > 0) {
+        ok = __all_sync(0xffffffffu, wait_bounded(bar_o + qi, (j - 1) & 1, w));
+        if (ok) {
+          tc_fence_after();
+          const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a frame with no valid list entry: zero output
+          const bool valid = row < r1;
+          __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * ltok + row) * p.HS + h) * D;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(o_tmem + 32 * c, o);
+            tmem_wait_ld_regs(o);
+            if (valid) {
+              uint4 pk[4];
+              uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pw[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+              uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// One CTA waits on a barrier that nothing arrives on; the bounded wait runs out.
+__global__ void watchdog_selftest_kernel(long long budget_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const Watch w{budget_cycles, &abort_flag};
+  (void)__all_sync(0xffffffffu, wait_bounded(&bar, 0, w));
+}
+
+__global__ void exp2_fma_eval_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (2 * i + 1 < n) {
+    const float2 r = exp2_fma2(make_float2(x[2 * i], x[2 * i + 1]));
+    y[2 * i] = r.x;
+    y[2 * i + 1] = r.y;
+  } else if (2 * i < n) {
+    y[2 * i] = exp2_fma2(make_float2(x[2 * i], 0.f)).x;
+  }
+}
+
+}  // namespace lvsa
