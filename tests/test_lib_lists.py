@@ -54,3 +54,14 @@ def test_errors(lib):
     buf = (ctypes.c_int32 * 10)()
     st = lib._lib.lvsa_build_frame_lists(8, 4, 2, 0, buf, 10, ctypes.byref(L))
     assert st == lib.LVSA_ERR_BUFFER_TOO_SMALL and L.value == 4
+
+
+def test_random_parameters_bit_exact(lib):
+    """Seeded random (T, C, W, step), including far steps and budgets at or above T."""
+    g = np.random.default_rng(2026)
+    for _ in range(300):
+        T = int(g.integers(1, 700))
+        C = int(g.integers(1, T + 3))
+        W = int(g.integers(1, C + 1))
+        s = int(g.integers(0, 10**9))
+        assert lib.lvsa_build_frame_lists(T, C, W, s).tolist() == OL.frame_lists(T, C, W, s), (T, C, W, s)
