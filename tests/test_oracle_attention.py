@@ -9,7 +9,8 @@ What pins what:
   frames are attended, each once; one dominant key -> its value row; adding a
   constant vector to every key changes nothing; list order does not matter;
 * T = 1 is ordinary attention over one frame;
-* planted mistakes (wrong scale, a frame counted twice, transposed product)
+* planted mistakes (wrong scale, a frame counted twice, transposed product, per-frame
+  softmax, frame tokens off by one, the previous frame's list)
   must fail one of the above.
 """
 
@@ -176,5 +177,57 @@ def test_mistake_transposed_product_is_caught(monkeypatch):
         return orig(k, q, v, lists, P, rows, scale)  # q and k swapped
 
     monkeypatch.setattr(OA, "sparse_attention_rows", transposed)
+    with pytest.raises(AssertionError):
+        test_sparse_matches_library_masked_attention(8, 5, 2, 8, 4, 2, 0)
+
+
+def test_mistake_per_frame_softmax_is_caught(monkeypatch):
+    """A softmax normalised within each frame (and the frames then averaged) instead of one joint softmax."""
+
+    def per_frame(q, k, v, lists, P, rows, scale=None):
+        B, _, H, d = np.shape(q)
+        q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+        sigma = OA.default_scale(d) if scale is None or scale <= 0 else scale
+        rows = np.asarray(list(rows))
+        out = np.zeros((B, rows.size, H, d))
+        for n, r in enumerate(rows):
+            frames = sorted(set(int(f) for f in lists[int(r) // P]))
+            for b in range(B):
+                for h in range(H):
+                    acc = np.zeros(d)
+                    for f in frames:
+                        toks = np.arange(f * P, (f + 1) * P)
+                        s = sigma * k[b, toks, h] @ q[b, r, h]
+                        e = np.exp(s - s.max())
+                        acc += (e / e.sum()) @ v[b, toks, h]
+                    out[b, n, h] = acc / len(frames)
+        return out
+
+    monkeypatch.setattr(OA, "sparse_attention_rows", per_frame)
+    with pytest.raises(AssertionError):
+        test_sparse_matches_library_masked_attention(8, 5, 2, 8, 4, 2, 0)
+
+
+def test_mistake_shifted_frame_tokens_is_caught(monkeypatch):
+    """Frame f's tokens taken one token late (an off-by-one in the gather)."""
+
+    def shifted(frames, P):
+        fs = sorted(set(int(f) for f in frames))
+        return np.concatenate([np.arange(f * P + 1, (f + 1) * P + 1) for f in fs]) % (8 * P)
+
+    monkeypatch.setattr(OA, "frame_tokens", shifted)
+    with pytest.raises(AssertionError):
+        test_sparse_matches_library_masked_attention(8, 5, 2, 8, 4, 2, 0)
+
+
+def test_mistake_previous_frame_list_is_caught(monkeypatch):
+    """Query rows of frame t given the list of frame t - 1."""
+    orig = OA.sparse_attention_rows
+
+    def prev_list(q, k, v, lists, P, rows, scale=None):
+        shifted = [lists[max(t - 1, 0)] for t in range(len(lists))]
+        return orig(q, k, v, shifted, P, rows, scale)
+
+    monkeypatch.setattr(OA, "sparse_attention_rows", prev_list)
     with pytest.raises(AssertionError):
         test_sparse_matches_library_masked_attention(8, 5, 2, 8, 4, 2, 0)
