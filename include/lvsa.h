@@ -117,6 +117,8 @@ lvsa_status lvsa_build_anchors(int T, int C, int W, long long step,
  * pipeline) stops that CTA, sets LVSA_DEV_TIMEOUT, and is reported by
  * lvsa_get_device_status after the stream is synchronised.
  * Needs an sm_100 (B200-class) device; otherwise LVSA_ERR_UNSUPPORTED.
+ * The call can be captured into a CUDA graph (the tensor maps travel by value
+ * in the launch parameters; a replay reads whatever the same buffers hold).
  */
 lvsa_status lvsa_attention(const void* q, const void* k, const void* v,
                            const int32_t* lists, int L, int T, int tokens_per_frame,
@@ -156,7 +158,8 @@ lvsa_status lvsa_attention(const void* q, const void* k, const void* v,
  *            lock while they are queued.
  * Behaviour: asynchronous; errors as lvsa_attention (a failure part-way
  * returns LVSA_ERR_CUDA and leaves out_host partly written).  Synchronise
- * `stream` before reading out_host.
+ * `stream` before reading out_host.  The call can be captured into a CUDA
+ * graph on `stream` (the internal streams join the capture through events).
  */
 lvsa_status lvsa_attention_host(const void* q_host, const void* k_host, const void* v_host,
                                 const int32_t* lists_host, int L, int T, int tokens_per_frame,

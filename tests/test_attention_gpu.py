@@ -347,3 +347,46 @@ def test_bench_json_line_contract():
     assert d["gpu_launches"] == 3
     for key in ("sm_mhz", "sm_max_mhz", "reasons"):
         assert key in d["clocks"], key
+
+
+def test_cuda_graph_capture_and_replay(gpu_lib):
+    """Both entry points can be captured into a CUDA graph (tensor maps travel by value in the launch
+    parameters; the host-buffer call's internal streams join the capture through its events); replays
+    give the eager results bit for bit, also after the inputs are changed in place."""
+    T, P, H, d = 6, 300, 3, 128
+    q, k, v = make(T, P, H, d, seed=41)
+    lists_np = gpu_lib.lvsa_build_frame_lists(T, 4, 2, 3)
+    lists = torch.from_numpy(lists_np).cuda()
+    out = torch.empty_like(q)
+    qh, kh, vh = (x.cpu().contiguous().pin_memory() for x in (q, k, v))
+    lh = torch.from_numpy(lists_np).pin_memory()
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    stage = [torch.empty_like(q) for _ in range(4)]
+    ld = torch.empty_like(lists)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up outside the capture (first-call setup)
+        gpu_lib.lvsa_attention(q, k, v, lists, P, out=out)
+        gpu_lib.lvsa_attention_host(qh, kh, vh, lh, P, oh, stage[0], stage[1], stage[2], ld, stage[3])
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1):
+        gpu_lib.lvsa_attention(q, k, v, lists, P, out=out)
+    with torch.cuda.graph(g2):
+        gpu_lib.lvsa_attention_host(qh, kh, vh, lh, P, oh, stage[0], stage[1], stage[2], ld, stage[3])
+    for trial in range(2):
+        if trial == 1:  # new inputs in the same buffers
+            q2, k2, v2 = make(T, P, H, d, seed=42)
+            q.copy_(q2), k.copy_(k2), v.copy_(v2)
+            qh.copy_(q2.cpu()), kh.copy_(k2.cpu()), vh.copy_(v2.cpu())
+        out.zero_()
+        oh.zero_()
+        torch.cuda.synchronize()
+        g1.replay()
+        g2.replay()
+        torch.cuda.synchronize()
+        eager = gpu_lib.lvsa_attention(q, k, v, lists, P)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+        assert torch.equal(oh.view(torch.int16), eager.cpu().view(torch.int16))
