@@ -230,6 +230,13 @@ def run_reference(args, rank, world):
     return 0
 
 
+def head_band(rank: int, world: int, H: int):
+    """Heads [h0, h0 + n) of rank `rank` when H heads are split as evenly as possible over `world` ranks."""
+    base, extra = divmod(H, world)
+    n = base + (1 if rank < extra else 0)
+    return rank * base + min(rank, extra), n
+
+
 def workload_config(w, world, fixed_grid=False):
     return {"workload": w.name, "anchors": "fixed grid (step 0 pattern every step)" if fixed_grid else "rotating", "T": w.T, "tokens_per_frame": w.P, "heads": w.H, "head_dim": w.d, "C": w.C,
             "W": w.W, "G": max(0, w.C - w.W) if w.C < w.T else 0, "global_batch": w.B * world,
@@ -248,8 +255,20 @@ def run_lvsa(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = synthetic.WORKLOADS[args.workload]
-    F = flops_per_call(w)
     q, k, v = synthetic.make_qkv(w, device=dev)
+    w_full, h0, hn = w, 0, w.H
+    shard = args.shard_heads and world > 1
+    if shard:
+        # one call split over the ranks by heads (heads are independent; the lists are shared): this rank
+        # computes heads [h0, h0 + hn) of the same synthetic tensors, nothing is exchanged
+        if world > w.H:
+            raise SystemExit(f"--shard-heads needs at most {w.H} ranks")
+        h0, hn = head_band(rank, world, w.H)
+        q, k, v = (x[:, :, h0:h0 + hn].contiguous() for x in (q, k, v))
+        w = synthetic.Workload(w.name, T=w.T, P=w.P, H=hn, d=w.d, C=w.C, W=w.W, B=w.B, seed=w.seed)
+    F = flops_per_call(w)            # this rank's kernel
+    F_call = flops_per_call(w_full)  # one whole call
+    calls = 1 if shard else world    # per step, over all ranks: sharded ranks share one call
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
     nsteps = args.warmup + args.steps
@@ -298,7 +317,7 @@ def run_lvsa(args, rank, world, local):
     if status:
         raise RuntimeError(f"device status {status:#x} after the timed region")
     ms_per_step = elapsed_ms / args.steps
-    value = world * F * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = calls * F_call * args.steps / (elapsed_ms * 1e-3) / 1e12
     if args.kernel_only:
         if rank == 0:
             print(json.dumps({"workload": w.name, "value": value, "unit": "TFLOP/s", "ms_per_step": ms_per_step,
@@ -350,11 +369,11 @@ def run_lvsa(args, rank, world, local):
     # ---------------------------------------------------------------- roofline of the kernel
     peaks, peak_src = load_peaks()
     kern_avg_ms = sum(kernel_ms) / len(kernel_ms)
-    achieved = F / (kern_avg_ms * 1e-3) / 1e12
+    achieved = F / (kern_avg_ms * 1e-3) / 1e12  # this rank's kernel (its heads when sharded)
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
+    if os.path.exists(tpath) and not shard:
         try:
             with open(tpath) as f:
                 tj = json.load(f)
@@ -365,9 +384,12 @@ def run_lvsa(args, rank, world, local):
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if shard else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w, world, args.fixed_grid),
+        "config": (dict(workload_config(w_full, 1, args.fixed_grid),
+                        parallelism=f"heads split over {world} ranks (this rank {h0}..{h0 + hn - 1})")
+                   if shard else workload_config(w, world, args.fixed_grid)),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 dense (burst)",
@@ -376,7 +398,8 @@ def run_lvsa(args, rank, world, local):
         "kernel_ms_over_steps": {"steps": f"s = {args.warmup}..{args.warmup + args.steps - 1}",
                                  "mean": kern_avg_ms, "median": statistics.median(kernel_ms),
                                  "min": min(kernel_ms), "max": max(kernel_ms)},
-        "e2e": {"value": F / (e2e_ms * 1e-3) / 1e12 * world, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": calls * F_call / (e2e_ms * 1e-3) / 1e12,
+                "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "call": "lvsa_attention_host (pinned host buffers; copies pipelined by bands of "
                         f"{args.heads_per_band or 1} head(s))"},
@@ -471,6 +494,9 @@ def main(argv=None):
     ap.add_argument("--kernel-only", action="store_true",
                     help="time the device path only and print a short line (for profiling runs)")
     ap.add_argument("--ref-seconds", type=float, default=0.0, help="reference arm: CPU seconds per step")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="with --gpus N > 1: split one call over the ranks by heads (strong scaling) "
+                         "instead of running a replica per rank")
     ap.add_argument("--heads-per-band", type=int, default=0,
                     help="end-to-end call: heads per pipelined band (0: one)")
     args = ap.parse_args(argv)

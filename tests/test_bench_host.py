@@ -92,3 +92,13 @@ def test_reference_arm_nonzero_rank_exits_without_work():
         ref_seconds = 0.01
 
     assert bench.run_reference(A, rank=1, world=2) == 0
+
+
+def test_head_bands_cover_every_head_once():
+    for H in range(1, 41):
+        for world in range(1, min(H, 8) + 1):
+            bands = [bench.head_band(r, world, H) for r in range(world)]
+            covered = [h for h0, n in bands for h in range(h0, h0 + n)]
+            assert covered == list(range(H))
+            sizes = [n for _, n in bands]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
