@@ -175,6 +175,8 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
     return LVSA_ERR_INVALID_ARG;
   const lvsa_status cs = check_sizes(L, T, P, heads, d, batch, scale);
   if (cs != LVSA_OK) return cs;
+  const size_t bytes = static_cast<size_t>(batch) * T * P * heads * static_cast<size_t>(d) * 2;
+  if (!disjoint(out, q, bytes) || !disjoint(out, k, bytes) || !disjoint(out, v, bytes)) return LVSA_ERR_INVALID_ARG;
   int dev = 0;
   const lvsa_status ds = check_device(&dev);
   if (ds != LVSA_OK) return ds;

@@ -109,7 +109,7 @@ lvsa_status lvsa_build_anchors(int T, int C, int W, long long step,
  *   T, tokens_per_frame (P), heads (H), d, batch: sizes; d must be 64 or 128;
  *            T <= 4096 (LVSA_ERR_UNSUPPORTED above).
  *   scale    softmax scale; <= 0 selects 1/sqrt(d).
- *   out      DEVICE bf16, same layout as q, 16-byte aligned, must not alias
+ *   out      DEVICE bf16, same layout as q, 16-byte aligned, must not overlap
  *            q, k or v.
  *   stream   a cudaStream_t (passed as void*), NULL = default stream.
  * Behaviour: asynchronous on `stream`; returns after the launch.  Argument and

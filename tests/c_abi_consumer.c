@@ -27,11 +27,14 @@ int main(void) {
   const lvsa_status sa = lvsa_build_anchors(8, 4, 2, 1, anchors, 2, &G);
   printf("anchors %s G=%d %d %d\n", lvsa_status_string(sa), G, (int)anchors[0], (int)anchors[1]);
   /* refused before any CUDA call */
-  printf("null q: %s\n", lvsa_status_string(lvsa_attention(NULL, (void*)16, (void*)32, (const int32_t*)48, 4, 8, 64,
-                                                           2, 64, 1, 0.0f, (void*)64, NULL)));
-  printf("d=96: %s\n", lvsa_status_string(lvsa_attention((void*)1024, (void*)2048, (void*)4096,
-                                                         (const int32_t*)8192, 4, 8, 64, 2, 96, 1, 0.0f,
-                                                         (void*)16384, NULL)));
+  /* fake, 16-byte aligned, non-overlapping addresses: validation fails before any is used */
+  const uintptr_t A = (uintptr_t)1 << 24, M = (uintptr_t)1 << 20;
+  printf("null q: %s\n", lvsa_status_string(lvsa_attention(NULL, (void*)(A + M), (void*)(A + 2 * M),
+                                                           (const int32_t*)(A + 3 * M), 4, 8, 64, 2, 64, 1, 0.0f,
+                                                           (void*)(A + 4 * M), NULL)));
+  printf("d=96: %s\n", lvsa_status_string(lvsa_attention((void*)A, (void*)(A + M), (void*)(A + 2 * M),
+                                                         (const int32_t*)(A + 3 * M), 4, 8, 64, 2, 96, 1, 0.0f,
+                                                         (void*)(A + 4 * M), NULL)));
   printf("small buffer: %s\n", lvsa_status_string(lvsa_build_frame_lists(8, 4, 2, 0, lists, 4, &L)));
   printf("version %d\n", lvsa_version());
   return 0;

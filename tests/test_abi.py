@@ -40,9 +40,10 @@ def test_status_strings(lib):
 
 
 def test_attention_argument_validation_without_gpu(lib):
-    A = 1 << 20  # a 16-byte aligned fake address; validation fails before it is used
-    good = dict(q=A, k=A + 4096, v=A + 8192, lists=A + 12288, L=4, T=8, P=64, H=2, d=64, B=1, scale=0.0,
-                out=A + 16384, stream=0)
+    A = 1 << 24  # 16-byte aligned fake addresses 1 MB apart (no overlap); validation fails before any is used
+    M = 1 << 20
+    good = dict(q=A, k=A + M, v=A + 2 * M, lists=A + 3 * M, L=4, T=8, P=64, H=2, d=64, B=1, scale=0.0,
+                out=A + 4 * M, stream=0)
 
     def call(**kw):
         a = dict(good, **kw)
@@ -60,8 +61,9 @@ def test_attention_argument_validation_without_gpu(lib):
     assert call(H=0) == INV
     assert call(B=0) == INV
     assert call(out=A) == INV            # aliases q
+    assert call(out=A + 64) == INV       # overlaps q (and k, v) without being equal
     assert call(q=A + 8) == INV          # not 16-byte aligned
-    assert call(lists=A + 12290) == INV  # int32 misaligned
+    assert call(lists=A + 3 * M + 2) == INV  # int32 misaligned
     assert call(scale=float("nan")) == INV
     assert call(T=1 << 20, P=1 << 12) == INV  # T*P overflows int32
     assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
