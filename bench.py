@@ -232,9 +232,9 @@ def run_reference(args, rank, world):
 
 def head_band(rank: int, world: int, H: int):
     """Heads [h0, h0 + n) of rank `rank` when H heads are split as evenly as possible over `world` ranks."""
-    base, extra = divmod(H, world)
-    n = base + (1 if rank < extra else 0)
-    return rank * base + min(rank, extra), n
+    from block_sparse_attention_frame_b200.sequence_parallel import head_band as band
+
+    return band(rank, world, H)
 
 
 def workload_config(w, world, fixed_grid=False):
@@ -461,6 +461,121 @@ def run_sweep(args, rank, world, local):
     return 0
 
 
+def run_sequence_parallel(args, rank, world, local):
+    """One call split over the ranks by token ranges (DeepSpeed-Ulysses layout, the pages' multi-device
+    setting): rank r holds tokens of Q, K, V and of the output for every head; its band of heads is gathered
+    from the other ranks by peer loads, and the attention stores each output row into its owner's buffer."""
+    import torch
+
+    import block_sparse_attention_frame_b200 as lvsa
+    from block_sparse_attention_frame_b200 import synthetic
+    from block_sparse_attention_frame_b200.sequence_parallel import SequenceParallelAttention
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = synthetic.WORKLOADS[args.workload]
+    if world > w.H:
+        raise SystemExit(f"--sequence-parallel needs at most {w.H} ranks")
+    sp = SequenceParallelAttention(w.T, w.P, w.H, w.d, batch=w.B, device=dev)
+    q, k, v = synthetic.make_qkv(w, device=dev)  # the same seeded tensors on every rank
+    a, b = sp.starts[rank], sp.starts[rank + 1]
+    for dst, src in ((sp.q, q), (sp.k, k), (sp.v, v)):
+        dst.copy_(src[:, a:b])
+    del q, k, v
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream(dev)
+    nsteps = args.warmup + args.steps
+    pinned = [torch.empty((w.T, w.L), dtype=torch.int32).pin_memory() for _ in range(nsteps)]
+    lists_dev = torch.empty((w.T, w.L), dtype=torch.int32, device=dev)
+
+    def step(s, events=None):
+        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=pinned[s % nsteps].numpy())
+        lists_dev.copy_(pinned[s % nsteps], non_blocking=True)
+        sp(lists_dev, events=events)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    events = []
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, events)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
+    gather_ms = [e0.elapsed_time(e1) for e0, e1, _ in events]
+    attn_ms = [e1.elapsed_time(e2) for _, e1, e2 in events]
+    if lvsa.lvsa_get_device_status(clear=True):
+        raise RuntimeError("device status set after the timed region")
+
+    # end to end: this rank's token range of Q, K, V from pinned host memory, its output rows back
+    qh, kh, vh = (x.cpu().pin_memory() for x in (sp.q, sp.k, sp.v))
+    oh = torch.empty(sp.out.shape, dtype=sp.out.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step(s):
+        for dst, src in ((sp.q, qh), (sp.k, kh), (sp.v, vh)):
+            dst.copy_(src, non_blocking=True)
+        step(s)
+        oh.copy_(sp.out, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+
+    F_call = flops_per_call(w)
+    F_band = 4.0 * w.B * sp.band * w.T * w.L * w.P * w.P * w.d
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    kern = sum(attn_ms) / len(attn_ms)
+    achieved = F_band / (kern * 1e-3) / 1e12 if sp.band else 0.0
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if world == 1 and os.path.exists(tpath):
+        with open(tpath) as f:
+            tj = json.load(f)
+        if tj.get("workload") == w.name and tj.get("kernel_source_hash") == kernel_source_hash():
+            traffic = tj.get("bytes_per_launch")
+    row_bytes = w.H * w.d * 2
+    peer_bytes = 3 * w.B * (w.T * w.P - (b - a)) * sp.band * w.d * 2 if world > 1 else 0
+    line = {
+        "metric": METRIC, "value": F_call * args.steps / (elapsed_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, 1), parallelism=(
+            f"sequence-parallel over {world} rank(s) (Ulysses layout): token ranges {sp.chunk_tokens}; "
+            f"this rank heads {sp.head0}..{sp.head0 + sp.band - 1}; heads gathered by peer loads, output rows "
+            "stored to their owners by the attention kernel")),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "kernel_ms_avg": kern, "flops_per_launch": F_band},
+        "exchange": {"gather_ms_avg": sum(gather_ms) / len(gather_ms), "peer_bytes_read_per_step": peer_bytes,
+                     "gather_GBps": (peer_bytes / (sum(gather_ms) / len(gather_ms) * 1e-3) / 1e9)
+                     if peer_bytes else None},
+        "e2e": {"value": F_call / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * w.B * (b - a) * row_bytes + w.T * w.L * 4,
+                "d2h_bytes_per_step": w.B * (b - a) * row_bytes,
+                "call": "SequenceParallelAttention on this rank's token range (pinned host buffers)"},
+        "gpu_launches": args.steps * (2 if world > 1 else 1),
+        "clocks": clocks.summary(),
+    }
+    sp.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def flops_per_call_dense(w) -> float:
     return 4.0 * w.B * w.H * w.T * w.T * w.P * w.P * w.d
 
@@ -497,6 +612,8 @@ def main(argv=None):
     ap.add_argument("--shard-heads", action="store_true",
                     help="with --gpus N > 1: split one call over the ranks by heads (strong scaling) "
                          "instead of running a replica per rank")
+    ap.add_argument("--sequence-parallel", action="store_true",
+                    help="split one call over the ranks by token ranges (Ulysses layout, peer-memory exchanges)")
     ap.add_argument("--heads-per-band", type=int, default=0,
                     help="end-to-end call: heads per pipelined band (0: one)")
     args = ap.parse_args(argv)
@@ -507,6 +624,8 @@ def main(argv=None):
             return run_reference(args, rank, world)
         if args.sweep:
             return run_sweep(args, rank, world, local)
+        if args.sequence_parallel:
+            return run_sequence_parallel(args, rank, world, local)
         return run_lvsa(args, rank, world, local)
     finally:
         if world > 1:

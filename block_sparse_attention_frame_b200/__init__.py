@@ -11,6 +11,10 @@ Functions carry the C ABI's names (declared in ``include/lvsa.h``):
 ``lvsa_attention(q, k, v, lists, tokens_per_frame, scale=0, out=None, stream=None)``
 ``lvsa_attention_host(q_host, k_host, v_host, lists_host, tokens_per_frame, out_host, q_dev, k_dev, v_dev,
 lists_dev, out_dev, scale=0, heads_per_band=0, stream=None)``
+``lvsa_seq_to_heads(q_chunks, k_chunks, v_chunks, chunk_tokens, head0, band, q_band, k_band, v_band, stream=None)``
+``lvsa_attention_to_chunks(q, k, v, lists, tokens_per_frame, out_chunks, chunk_tokens, out_heads, head0, scale=0,
+stream=None)``
+``lvsa_ipc_export(tensor)`` -> bytes, ``lvsa_ipc_import(handle)`` -> int, ``lvsa_ipc_release(ptr)``
 ``lvsa_get_device_status(clear=False)``   -> int (LVSA_DEV_* bits)
 ``lvsa_set_wait_budget_ns(ns)``, ``lvsa_watchdog_selftest(budget_ns, stream=None)``
 """
@@ -34,11 +38,13 @@ LVSA_ERR_BUFFER_TOO_SMALL = 5
 LVSA_ERR_BAD_LIST = 6
 LVSA_DEV_TIMEOUT = 0x1
 LVSA_DEV_BAD_LIST = 0x2
+LVSA_IPC_HANDLE_BYTES = 72
 
 EXPORTED = [
     "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_attention_host", "lvsa_get_device_status",
     "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_exp2_fma_eval", "lvsa_status_string",
-    "lvsa_version",
+    "lvsa_version", "lvsa_seq_to_heads", "lvsa_attention_to_chunks", "lvsa_ipc_export", "lvsa_ipc_import",
+    "lvsa_ipc_release",
 ]
 
 
@@ -68,6 +74,18 @@ _lib.lvsa_attention.restype = _c_int
 _lib.lvsa_attention_host.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_vp]
 _lib.lvsa_attention_host.restype = _c_int
+_lib.lvsa_seq_to_heads.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                   _c_vp, _c_vp, _c_vp, _c_vp]
+_lib.lvsa_seq_to_heads.restype = _c_int
+_lib.lvsa_attention_to_chunks.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                          _c_float, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_vp]
+_lib.lvsa_attention_to_chunks.restype = _c_int
+_lib.lvsa_ipc_export.argtypes = [_c_vp, _c_vp]
+_lib.lvsa_ipc_export.restype = _c_int
+_lib.lvsa_ipc_import.argtypes = [_c_vp, ctypes.POINTER(_c_vp)]
+_lib.lvsa_ipc_import.restype = _c_int
+_lib.lvsa_ipc_release.argtypes = [_c_vp]
+_lib.lvsa_ipc_release.restype = _c_int
 _lib.lvsa_get_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), _c_int]
 _lib.lvsa_get_device_status.restype = _c_int
 _lib.lvsa_set_wait_budget_ns.argtypes = [_c_ull]
@@ -219,6 +237,118 @@ def lvsa_attention_host_raw(*args) -> int:
     a[10] = float(a[10])
     a[18] = ctypes.c_void_p(a[18])
     return int(_lib.lvsa_attention_host(*a))
+
+
+def _addr(x) -> int:
+    """A device address: a CUDA tensor's data pointer, or an int (e.g. from lvsa_ipc_import); 0 for None."""
+    if x is None:
+        return 0
+    return int(x.data_ptr()) if hasattr(x, "data_ptr") else int(x)
+
+
+def _ptr_table(xs):
+    return (ctypes.c_void_p * len(xs))(*[_addr(x) or None for x in xs])
+
+
+def _int_table(xs):
+    return (ctypes.c_int * len(xs))(*[int(x) for x in xs])
+
+
+def lvsa_seq_to_heads_raw(q_chunks, k_chunks, v_chunks, chunk_tokens, heads: int, head0: int, band: int, d: int,
+                          batch: int, q_band, k_band, v_band, stream_ptr: int = 0) -> int:
+    """The C call (pointer tables as Python sequences of addresses); returns the status unchanged."""
+    n = len(chunk_tokens)
+    return int(_lib.lvsa_seq_to_heads(_ptr_table(q_chunks), _ptr_table(k_chunks), _ptr_table(v_chunks),
+                                      _int_table(chunk_tokens), n, heads, head0, band, d, batch, _addr(q_band),
+                                      _addr(k_band), _addr(v_band), ctypes.c_void_p(stream_ptr)))
+
+
+def lvsa_seq_to_heads(q_chunks, k_chunks, v_chunks, chunk_tokens, head0: int, band: int, q_band, k_band, v_band,
+                      heads: int | None = None, stream=None):
+    """Gather heads [head0, head0 + band) of Q, K, V from token-range buffers (this GPU's tensors or peer
+    addresses) into the whole-sequence band buffers q_band, k_band, v_band [batch, tokens, band, d].
+    ``heads``: heads per row of the range buffers (taken from the first range that is a tensor if None)."""
+    import torch
+
+    for name, x in (("q_band", q_band), ("k_band", k_band), ("v_band", v_band)):
+        if not isinstance(x, torch.Tensor) or x.device.type != "cuda" or x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+        if not x.is_contiguous() or x.dim() != 4 or x.shape != q_band.shape:
+            raise ValueError(f"{name} must be contiguous [batch, tokens, band, d] shaped like q_band")
+    B, ntok, nb, d = q_band.shape
+    if nb != band or ntok != sum(int(c) for c in chunk_tokens):
+        raise ValueError("q_band must be [batch, sum(chunk_tokens), band, d]")
+    if heads is None:
+        ts = [x for x in list(q_chunks) if isinstance(x, torch.Tensor)]
+        if not ts:
+            raise ValueError("heads must be given when no range buffer is a tensor")
+        heads = ts[0].shape[2]
+    with torch.cuda.device(q_band.device):
+        st = lvsa_seq_to_heads_raw(q_chunks, k_chunks, v_chunks, chunk_tokens, heads, head0, band, d, B, q_band,
+                                   k_band, v_band, _stream_ptr(stream, q_band.device).value or 0)
+    _check("lvsa_seq_to_heads", st)
+
+
+def lvsa_attention_to_chunks_raw(q, k, v, lists, L: int, T: int, P: int, heads: int, d: int, batch: int,
+                                 scale: float, out_chunks, chunk_tokens, out_heads: int, head0: int,
+                                 stream_ptr: int = 0) -> int:
+    """The C call (pointer tables as Python sequences of addresses); returns the status unchanged."""
+    return int(_lib.lvsa_attention_to_chunks(_addr(q), _addr(k), _addr(v), _addr(lists), L, T, P, heads, d, batch,
+                                             float(scale), _ptr_table(out_chunks), _int_table(chunk_tokens),
+                                             len(chunk_tokens), out_heads, head0, ctypes.c_void_p(stream_ptr)))
+
+
+def lvsa_attention_to_chunks(q, k, v, lists, tokens_per_frame: int, out_chunks, chunk_tokens, out_heads: int,
+                             head0: int, scale: float = 0.0, stream=None):
+    """Block-sparse attention of the heads of q, k, v [batch, T*P, heads, d], each output row stored into the
+    token-range buffer that holds its token: out_chunks[c] [batch, chunk_tokens[c], out_heads, d] (tensors on
+    this GPU or peer addresses), heads head0 .. head0 + heads - 1."""
+    import torch
+
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(x, torch.Tensor) or x.device.type != "cuda" or x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+        if not x.is_contiguous() or x.dim() != 4 or x.shape != q.shape:
+            raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q")
+    if lists.device.type != "cuda" or lists.dtype != torch.int32 or lists.dim() != 2 or not lists.is_contiguous():
+        raise TypeError("lists must be a contiguous CUDA int32 tensor [T, L]")
+    if len(out_chunks) != len(chunk_tokens):
+        raise ValueError("one token count per output buffer")
+    for x, n in zip(out_chunks, chunk_tokens):
+        if isinstance(x, torch.Tensor) and (x.dtype != torch.bfloat16 or not x.is_contiguous() or x.dim() != 4
+                                            or x.shape[1:] != (n, out_heads, q.shape[3])):
+            raise ValueError("an output buffer tensor must be contiguous bf16 [batch, tokens of its range, "
+                             "out_heads, d]")
+    B, ntok, H, d = q.shape
+    T, L = lists.shape
+    if ntok != T * tokens_per_frame:
+        raise ValueError(f"q has {ntok} tokens, expected T*tokens_per_frame = {T * tokens_per_frame}")
+    with torch.cuda.device(q.device):
+        st = lvsa_attention_to_chunks_raw(q, k, v, lists, L, T, tokens_per_frame, H, d, B, scale, out_chunks,
+                                          chunk_tokens, out_heads, head0,
+                                          _stream_ptr(stream, q.device).value or 0)
+    _check("lvsa_attention_to_chunks", st)
+
+
+def lvsa_ipc_export(x) -> bytes:
+    """IPC handle (LVSA_IPC_HANDLE_BYTES bytes) of the device buffer holding tensor/address ``x``."""
+    buf = ctypes.create_string_buffer(LVSA_IPC_HANDLE_BYTES)
+    _check("lvsa_ipc_export", _lib.lvsa_ipc_export(_addr(x), buf))
+    return buf.raw
+
+
+def lvsa_ipc_import(handle: bytes) -> int:
+    """Maps another process's exported buffer on the current device; returns its address here."""
+    if len(handle) != LVSA_IPC_HANDLE_BYTES:
+        raise ValueError(f"an IPC handle has {LVSA_IPC_HANDLE_BYTES} bytes")
+    ptr = ctypes.c_void_p(0)
+    _check("lvsa_ipc_import", _lib.lvsa_ipc_import(ctypes.create_string_buffer(handle, len(handle)),
+                                                   ctypes.byref(ptr)))
+    return int(ptr.value)
+
+
+def lvsa_ipc_release(ptr: int) -> None:
+    _check("lvsa_ipc_release", _lib.lvsa_ipc_release(ctypes.c_void_p(int(ptr))))
 
 
 def lvsa_get_device_status(clear: bool = False) -> int:

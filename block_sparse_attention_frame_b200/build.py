@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "liblvsa.so")
 
-SOURCES = ["lists.cpp", "attention.cu"]
+SOURCES = ["lists.cpp", "attention.cu", "exchange.cu"]
 HEADERS = [os.path.join(INCLUDE, "lvsa.h"), os.path.join(CSRC, "sm100.cuh"), os.path.join(CSRC, "attention_kernel.cuh")]
 
 

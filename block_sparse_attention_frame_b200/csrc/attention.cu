@@ -92,11 +92,30 @@ lvsa_status check_device(int* dev) {
   return major == 10 ? LVSA_OK : LVSA_ERR_UNSUPPORTED;
 }
 
-// One launch over `heads` heads whose rows hold `head_stride` heads; q, k, v, out point
-// at the band's first head.  Arguments are already validated.
+// Where a launch writes its output: token ranges of the frame-major sequence, one buffer each, every
+// buffer [batch][tokens of its range][head_stride][d], this launch's heads starting at head0.
+struct Route {
+  int nchunks = 1;
+  int start[kMaxChunks + 1] = {};
+  void* out[kMaxChunks] = {};
+  int head_stride = 1;
+  int head0 = 0;
+  int routed = 0;
+};
+
+Route one_buffer(void* out, long long tokens, int head_stride) {
+  Route r;
+  r.start[1] = static_cast<int>(tokens);
+  r.out[0] = out;
+  r.head_stride = head_stride;
+  return r;
+}
+
+// One launch over `heads` heads whose input rows hold `in_stride` heads; q, k, v point at the band's
+// first head.  Arguments are already validated.
 lvsa_status launch_band(const void* q, const void* k, const void* v, const int32_t* lists, int L, int T, int P,
-                        int heads, int head_stride, int d, int batch, float scale, void* out, cudaStream_t st,
-                        int dev) {
+                        int heads, int in_stride, int d, int batch, float scale, const Route& route,
+                        cudaStream_t st, int dev) {
   const int qblocks = (P + kQTiles * kBM - 1) / (kQTiles * kBM);
   // frames of at least 256 tokens: query blocks of 256 rows run over the whole
   // sequence (a block may hold the end of one frame and the start of the next);
@@ -107,16 +126,21 @@ lvsa_status launch_band(const void* q, const void* k, const void* v, const int32
   if (nblocks > INT_MAX) return LVSA_ERR_INVALID_ARG;
   KernelParams kp;
   const long long tokens = static_cast<long long>(T) * P;
-  if (!make_map(&kp.tm_q, q, batch, tokens, heads, head_stride, d) ||
-      !make_map(&kp.tm_k, k, batch, tokens, heads, head_stride, d) ||
-      !make_map(&kp.tm_v, v, batch, tokens, heads, head_stride, d))
+  if (!make_map(&kp.tm_q, q, batch, tokens, heads, in_stride, d) ||
+      !make_map(&kp.tm_k, k, batch, tokens, heads, in_stride, d) ||
+      !make_map(&kp.tm_v, v, batch, tokens, heads, in_stride, d))
     return LVSA_ERR_CUDA;
-  kp.out = static_cast<__nv_bfloat16*>(out);
   kp.lists = lists;
   kp.T = T;
   kp.P = P;
   kp.H = heads;
-  kp.HS = head_stride;
+  kp.HS = route.head_stride;
+  kp.head0 = route.head0;
+  kp.nchunks = route.nchunks;
+  kp.routed = route.routed;
+  for (int c = 0; c <= kMaxChunks; ++c) kp.chunk_start[c] = route.start[c <= route.nchunks ? c : route.nchunks];
+  for (int c = 0; c < kMaxChunks; ++c)
+    kp.out_chunk[c] = static_cast<__nv_bfloat16*>(c < route.nchunks ? route.out[c] : nullptr);
   kp.L = L;
   kp.qblocks = qblocks;
   kp.straddle = straddle;
@@ -180,7 +204,58 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   int dev = 0;
   const lvsa_status ds = check_device(&dev);
   if (ds != LVSA_OK) return ds;
-  return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale, out, static_cast<cudaStream_t>(stream),
+  return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale,
+                     one_buffer(out, static_cast<long long>(T) * P, heads), static_cast<cudaStream_t>(stream), dev);
+}
+
+extern "C" lvsa_status lvsa_attention_to_chunks(const void* q, const void* k, const void* v, const int32_t* lists,
+                                                int L, int T, int tokens_per_frame, int heads, int d, int batch,
+                                                float scale, void* const* out_chunks, const int* chunk_tokens,
+                                                int nchunks, int out_heads, int head0, void* stream) {
+  using namespace lvsa;
+  const int P = tokens_per_frame;
+  if (!q || !k || !v || !lists || !out_chunks || !chunk_tokens) return LVSA_ERR_INVALID_ARG;
+  if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T) return LVSA_ERR_INVALID_ARG;
+  if (nchunks < 1 || nchunks > kMaxChunks) return LVSA_ERR_INVALID_ARG;
+  if (head0 < 0 || out_heads < 1 || head0 + heads > out_heads || out_heads > 65535) return LVSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(lists) & 3u))
+    return LVSA_ERR_INVALID_ARG;
+  const lvsa_status cs = check_sizes(L, T, P, heads, d, batch, scale);
+  if (cs != LVSA_OK) return cs;
+  Route route;
+  route.nchunks = nchunks;
+  route.head_stride = out_heads;
+  route.head0 = head0;
+  long long tokens = 0;
+  const size_t in_bytes = static_cast<size_t>(batch) * T * P * heads * static_cast<size_t>(d) * 2;
+  for (int c = 0; c < nchunks; ++c) {
+    if (chunk_tokens[c] < 0) return LVSA_ERR_INVALID_ARG;
+    route.start[c] = static_cast<int>(tokens);
+    tokens += chunk_tokens[c];
+    if (tokens > static_cast<long long>(T) * P) return LVSA_ERR_INVALID_ARG;
+    route.out[c] = out_chunks[c];
+    if (chunk_tokens[c] == 0) continue;
+    if (!out_chunks[c] || !aligned16(out_chunks[c])) return LVSA_ERR_INVALID_ARG;
+    const size_t cb = static_cast<size_t>(batch) * chunk_tokens[c] * out_heads * static_cast<size_t>(d) * 2;
+    const uintptr_t o = reinterpret_cast<uintptr_t>(out_chunks[c]);
+    for (const void* in : {q, k, v}) {
+      const uintptr_t x = reinterpret_cast<uintptr_t>(in);
+      if (!(o + cb <= x || x + in_bytes <= o)) return LVSA_ERR_INVALID_ARG;
+    }
+  }
+  if (tokens != static_cast<long long>(T) * P) return LVSA_ERR_INVALID_ARG;
+  route.start[nchunks] = static_cast<int>(tokens);
+  int dev = 0;
+  const lvsa_status ds = check_device(&dev);
+  if (ds != LVSA_OK) return ds;
+  // a buffer in another GPU's memory (a peer mapping): its stores are released at system scope
+  for (int c = 0; c < nchunks; ++c) {
+    if (chunk_tokens[c] == 0) continue;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, out_chunks[c]) != cudaSuccess) return LVSA_ERR_INVALID_ARG;
+    if (at.type != cudaMemoryTypeDevice || at.device != dev) route.routed = 1;
+  }
+  return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale, route, static_cast<cudaStream_t>(stream),
                      dev);
 }
 
@@ -245,7 +320,7 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
     cudaStream_t ks = hp->k[gi & 1];
     if (!ok(cudaEventRecord(ev_in, hp->h2d)) || !ok(cudaStreamWaitEvent(ks, ev_in, 0))) return LVSA_ERR_CUDA;
     r = launch_band(dst[0] + off, dst[1] + off, dst[2] + off, lists_dev, L, T, P, hn, heads, d, batch, scale,
-                    static_cast<char*>(out_dev) + off, ks, dev);
+                    one_buffer(static_cast<char*>(out_dev) + off, static_cast<long long>(T) * P, heads), ks, dev);
     if (r != LVSA_OK) return r;
     if (!ok(cudaEventRecord(ev_k, ks)) || !ok(cudaStreamWaitEvent(hp->d2h, ev_k, 0))) return LVSA_ERR_CUDA;
     if (!ok(cudaMemcpy2DAsync(static_cast<char*>(out_host) + off, row_bytes, static_cast<const char*>(out_dev) + off,

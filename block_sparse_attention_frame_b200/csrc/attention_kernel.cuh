@@ -19,7 +19,10 @@
 //               online softmax in the exp2 domain with a lazily updated running max (O in TMEM is
 //               rescaled only when the max grows by more than 2^8), P written back over the S columns
 //               as bf16; rows of the other frame skip the tiles their frame does not attend.
-//               Epilogue O / l -> bf16 -> HBM.
+//               Epilogue O / l -> bf16 -> HBM.  The output rows may be split by token range over several
+//               buffers, other GPUs' included (sequence-parallel use): each row is stored straight into
+//               the buffer of the rank that owns its tokens, so the attention and the head-to-sequence
+//               exchange after it are one kernel.
 // Every wait is bounded: when its time budget runs out the CTA stops, sets a device status bit, lets its
 // in-flight copies and MMAs finish and frees TMEM.
 #pragma once
@@ -56,6 +59,7 @@ constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the max grows b
 constexpr int kPolyEvery = 0;             // every kPolyEvery-th element pair takes the FMA-pipe exp2 (0: none)
 
 constexpr int kMaxT = 4096;               // latent frames supported (frame bitmaps in shared memory)
+constexpr int kMaxChunks = 64;            // output buffers a launch can route rows to (token ranges)
 constexpr int kMapWords = kMaxT / 32;
 
 template <int D>
@@ -77,10 +81,14 @@ struct KernelParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
-  __nv_bfloat16* out;
   const int32_t* lists;
   int T, P, H, L;    // H: heads in this launch (grid.y)
-  int HS;            // heads per token row in memory (H for a whole tensor, more for a band of heads)
+  int HS;            // heads per token row of an output buffer (H for a whole tensor, more for a band)
+  int head0;         // output head of this launch's head 0 within such a row
+  int nchunks;       // output rows are split by token range over nchunks buffers
+  int routed;        // 1: some output buffers are another GPU's memory (stores released at system scope)
+  int chunk_start[kMaxChunks + 1];           // buffer c holds tokens [chunk_start[c], chunk_start[c + 1])
+  __nv_bfloat16* out_chunk[kMaxChunks];      // of every batch entry: [batch][tokens of c][HS][d]
   int straddle;      // 1: CTA c takes query rows [256c, 256c+256) of the whole frame-major sequence
   int qblocks;       // straddle == 0: ceil(P / 256) CTAs per query frame
   int nblocks;       // CTAs per (batch, head)
@@ -601,7 +609,16 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
           tc_fence_after();
           const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a frame with no valid list entry: zero output
           const bool valid = row < r1;
-          __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * ltok + row) * p.HS + h) * D;
+          // the buffer that holds this row's token: the last chunk starting at or before it (an empty
+          // chunk is never that one, since the next chunk starts at the same token)
+          int c = 0;
+          for (int hi = p.nchunks - 1; c < hi;) {
+            const int mid = (c + hi + 1) >> 1;
+            if (p.chunk_start[mid] <= row) c = mid; else hi = mid - 1;
+          }
+          const int c0 = p.chunk_start[c];
+          const size_t clen = static_cast<size_t>(p.chunk_start[c + 1] - c0);
+          __nv_bfloat16* dst = p.out_chunk[c] + ((b * clen + (row - c0)) * p.HS + p.head0 + h) * D;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
@@ -617,6 +634,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
               for (int i = 0; i < 4; ++i) d4[i] = pk[i];
             }
           }
+          // stores into another GPU's memory: ordered before anything the host does after this kernel
+          if (p.routed) __threadfence_system();
         }
       }
     }

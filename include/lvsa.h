@@ -17,7 +17,8 @@
  *  - Arguments are validated before any CUDA call or launch; on an error return
  *    no output has been written and nothing was launched.
  *  - The library never allocates device memory and never frees caller memory:
- *    the caller owns every buffer it passes.
+ *    the caller owns every buffer it passes (lvsa_ipc_import maps another
+ *    process's buffer; lvsa_ipc_release unmaps it).
  *  - Thread safety: lvsa_build_frame_lists is pure; lvsa_attention and
  *    lvsa_attention_host may be called from several host threads.
  */
@@ -166,6 +167,109 @@ lvsa_status lvsa_attention_host(const void* q_host, const void* k_host, const vo
                                 int heads, int d, int batch, float scale, void* out_host,
                                 void* q_dev, void* k_dev, void* v_dev, int32_t* lists_dev,
                                 void* out_dev, int heads_per_band, void* stream);
+
+/*
+ * Sequence-parallel use (DeepSpeed-Ulysses layout, under which the method runs
+ * Wan 2.2-A14B on 8 NPUs: techwalker article, section 五).  N ranks, one per
+ * GPU of a node; rank r holds tokens [start_r, start_r + n_r) of the
+ * frame-major sequence (n_r = chunk_tokens[r], start_r their prefix sum) of
+ * Q, K, V and the output, for every head: [batch][n_r][heads][d] bf16.  Rank r
+ * computes attention for a band of heads [head0, head0 + band) over all
+ * tokens -- heads are independent because A(t) is shared by every head (gist.science
+ * summary, section 2 "Core Mechanism").  Per step:
+ *   1. barrier (every rank's inputs written);
+ *   2. lvsa_seq_to_heads: gather the band from every rank's range, reading
+ *      the other GPUs' buffers through peer mappings (lvsa_ipc_import);
+ *   3. lvsa_attention_to_chunks: attention over the band, each output row
+ *      stored straight into the range buffer of the rank that owns its token;
+ *   4. barrier (every rank's output rows stored).
+ * No kernel of this library waits on another GPU; the caller's process group
+ * orders the ranks.
+ */
+
+/*
+ * lvsa_seq_to_heads -- gathers heads [head0, head0 + band) of Q, K and V from
+ * token-range buffers into whole-sequence band buffers (a pure copy, bit for
+ * bit).
+ *
+ * Arguments:
+ *   q_chunks, k_chunks, v_chunks  HOST arrays of nchunks DEVICE pointers (this
+ *            GPU's memory or a peer mapping), chunk c = [batch][chunk_tokens[c]]
+ *            [heads][d] bf16, 16-byte aligned; may be NULL where
+ *            chunk_tokens[c] == 0.
+ *   chunk_tokens  HOST int array of nchunks token counts (>= 0, sum >= 1);
+ *            ranges follow one another in array order.
+ *   nchunks  1..64.   heads, head0, band: 0 <= head0, 1 <= band,
+ *            head0 + band <= heads.   d: 64 or 128.   batch: 1..21845.
+ *   q_band, k_band, v_band  DEVICE bf16 [batch][sum of chunk_tokens][band][d],
+ *            16-byte aligned, pairwise disjoint and disjoint from every local
+ *            range buffer.
+ *   stream   a cudaStream_t (as void*).
+ * Behaviour: asynchronous; one launch for the three tensors.  The caller makes
+ * sure the range buffers are written (and not rewritten) while it runs.
+ */
+lvsa_status lvsa_seq_to_heads(const void* const* q_chunks, const void* const* k_chunks,
+                              const void* const* v_chunks, const int* chunk_tokens, int nchunks,
+                              int heads, int head0, int band, int d, int batch,
+                              void* q_band, void* k_band, void* v_band, void* stream);
+
+/*
+ * lvsa_attention_to_chunks -- lvsa_attention over a band of heads whose output
+ * rows go to token-range buffers: row i of the sequence is stored into the
+ * buffer c with start_c <= i < start_c + chunk_tokens[c], at token i - start_c
+ * and head head0 + h of its rows of out_heads heads.  The same arithmetic as
+ * lvsa_attention: the stored values are bit for bit those lvsa_attention
+ * writes for the same heads.
+ *
+ * Arguments:
+ *   q, k, v, lists, L, T, tokens_per_frame, heads, d, batch, scale  as
+ *            lvsa_attention (q, k, v: [batch][T*P][heads][d], e.g. the band
+ *            buffers of lvsa_seq_to_heads).
+ *   out_chunks  HOST array of nchunks DEVICE pointers (this GPU's memory or a
+ *            peer mapping), buffer c = [batch][chunk_tokens[c]][out_heads][d]
+ *            bf16, 16-byte aligned, disjoint from q, k, v; may be NULL where
+ *            chunk_tokens[c] == 0.  Heads outside [head0, head0 + heads) are
+ *            not written.
+ *   chunk_tokens  HOST int array, >= 0 each, summing to T * tokens_per_frame.
+ *   nchunks  1..64.   out_heads, head0: head0 >= 0, head0 + heads <= out_heads.
+ *   stream   a cudaStream_t (as void*).
+ * Behaviour: asynchronous; errors as lvsa_attention.  When a buffer is not
+ * this GPU's memory the kernel releases its stores at system scope before it
+ * ends, so the owner sees them once it has synchronised with this rank after
+ * the kernel (stream synchronisation, then a barrier).
+ */
+lvsa_status lvsa_attention_to_chunks(const void* q, const void* k, const void* v,
+                                     const int32_t* lists, int L, int T, int tokens_per_frame,
+                                     int heads, int d, int batch, float scale,
+                                     void* const* out_chunks, const int* chunk_tokens, int nchunks,
+                                     int out_heads, int head0, void* stream);
+
+/* Bytes of an IPC handle written by lvsa_ipc_export. */
+#define LVSA_IPC_HANDLE_BYTES 72
+
+/*
+ * lvsa_ipc_export -- writes an LVSA_IPC_HANDLE_BYTES handle for the device
+ * buffer holding dev_ptr (a CUDA IPC handle of its allocation plus the offset
+ * of dev_ptr in it) into the HOST buffer `handle`, for another process to map.
+ * dev_ptr must come from cudaMalloc (directly or through a caching allocator
+ * that uses it); memory from the virtual-memory API cannot be exported this
+ * way (LVSA_ERR_CUDA).  Errors: LVSA_ERR_INVALID_ARG (NULL, not device memory).
+ */
+lvsa_status lvsa_ipc_export(const void* dev_ptr, void* handle);
+
+/*
+ * lvsa_ipc_import -- maps the buffer of a handle written by lvsa_ipc_export in
+ * ANOTHER process (the same process cannot map its own handles) into this
+ * process on the current device, with peer access enabled when the buffer is
+ * on another GPU, and returns the pointer to use in *dev_ptr.  Mappings of the
+ * same allocation are shared and counted; release each pointer once.
+ */
+lvsa_status lvsa_ipc_import(const void* handle, void** dev_ptr);
+
+/* lvsa_ipc_release -- drops a pointer returned by lvsa_ipc_import (the mapping
+ * is closed with the last pointer into it).  LVSA_ERR_INVALID_ARG for a pointer
+ * that lvsa_ipc_import did not return or that was already released. */
+lvsa_status lvsa_ipc_release(void* dev_ptr);
 
 /*
  * lvsa_get_device_status -- device status bits (LVSA_DEV_*) of the current

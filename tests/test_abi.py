@@ -105,3 +105,74 @@ def test_host_path_argument_validation_without_gpu(lib):
 
     if not cuda_available():
         assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
+
+
+def test_seq_to_heads_argument_validation_without_gpu(lib):
+    A, M = 1 << 24, 1 << 20  # fake 16-byte aligned addresses 1 MB apart
+    good = dict(q=[A, A + M], k=[A + 2 * M, A + 3 * M], v=[A + 4 * M, A + 5 * M], n=[64, 64], H=4, h0=1, band=2,
+                d=64, B=1, qb=A + 8 * M, kb=A + 9 * M, vb=A + 10 * M)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return lib.lvsa_seq_to_heads_raw(a["q"], a["k"], a["v"], a["n"], a["H"], a["h0"], a["band"], a["d"], a["B"],
+                                         a["qb"], a["kb"], a["vb"])
+
+    INV = lib.LVSA_ERR_INVALID_ARG
+    assert call(q=[0, A + M]) == INV              # a range with tokens needs a buffer
+    assert call(q=[0, A + M], n=[0, 128]) != INV  # ... an empty one does not
+    assert call(q=[A + 8, A + M]) == INV          # misaligned source
+    assert call(qb=A + 8 * M + 8) == INV          # misaligned destination
+    assert call(n=[-1, 64]) == INV
+    assert call(n=[0, 0]) == INV                  # no token at all
+    assert call(h0=3) == INV                      # band past the last head
+    assert call(band=0) == INV
+    assert call(h0=-1) == INV
+    assert call(B=0) == INV
+    assert call(kb=A + 8 * M) == INV              # two band buffers overlap
+    assert call(qb=A + M) == INV                  # a band buffer overlaps a local range buffer
+    assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
+    assert lib.lvsa_seq_to_heads_raw([A] * 65, [A] * 65, [A] * 65, [1] * 65, 4, 0, 1, 64, 1, A + 8 * M, A + 9 * M,
+                                     A + 10 * M) == INV  # more ranges than a launch takes
+    assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)  # valid: fails only at the CUDA step
+
+
+def test_attention_to_chunks_argument_validation_without_gpu(lib):
+    A, M = 1 << 24, 1 << 20
+    T, P, H, d = 8, 64, 2, 64
+    good = dict(q=A, k=A + M, v=A + 2 * M, lists=A + 3 * M, L=4, T=T, P=P, H=H, d=d, B=1, scale=0.0,
+                outs=[A + 4 * M, A + 5 * M, A + 6 * M], n=[100, 0, T * P - 100], out_heads=4, h0=2)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return lib.lvsa_attention_to_chunks_raw(a["q"], a["k"], a["v"], a["lists"], a["L"], a["T"], a["P"], a["H"],
+                                                a["d"], a["B"], a["scale"], a["outs"], a["n"], a["out_heads"],
+                                                a["h0"])
+
+    INV = lib.LVSA_ERR_INVALID_ARG
+    assert call(n=[100, 0, T * P - 101]) == INV     # ranges must cover the sequence exactly
+    assert call(n=[100, 0, T * P]) == INV
+    assert call(n=[100, -1, T * P - 99]) == INV
+    assert call(outs=[0, A + 5 * M, A + 6 * M]) == INV  # a non-empty range needs a buffer
+    assert call(outs=[A + 4 * M, 0, A + 6 * M]) != INV  # an empty range does not
+    assert call(outs=[A + 4 * M + 8, A + 5 * M, A + 6 * M]) == INV
+    assert call(outs=[A + 4 * M, A + 5 * M, A + 2 * M]) == INV  # an output buffer overlaps v
+    assert call(h0=3) == INV                        # heads past out_heads
+    assert call(out_heads=1) == INV
+    assert call(h0=-1) == INV
+    assert call(outs=[A + 4 * M] * 65, n=[T * P] + [0] * 64) == INV  # more ranges than a launch takes
+    assert call(q=0) == INV
+    assert call(L=9) == INV
+    assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
+    assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
+
+
+def test_ipc_calls_reject_null_and_unknown_pointers(lib):
+    import ctypes
+
+    assert lib._lib.lvsa_ipc_export(None, ctypes.create_string_buffer(lib.LVSA_IPC_HANDLE_BYTES)) == \
+        lib.LVSA_ERR_INVALID_ARG
+    assert lib._lib.lvsa_ipc_import(None, ctypes.byref(ctypes.c_void_p())) == lib.LVSA_ERR_INVALID_ARG
+    assert lib._lib.lvsa_ipc_release(None) == lib.LVSA_ERR_INVALID_ARG
+    assert lib._lib.lvsa_ipc_release(ctypes.c_void_p(1 << 24)) == lib.LVSA_ERR_INVALID_ARG  # never imported
+    with pytest.raises(ValueError):
+        lib.lvsa_ipc_import(b"short")
