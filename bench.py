@@ -570,10 +570,47 @@ def run_sequence_parallel(args, rank, world, local):
         "gpu_launches": args.steps * (2 if world > 1 else 1),
         "clocks": clocks.summary(),
     }
+    if world == 1 and w.B == 1:
+        line["exchange"]["gather_local"] = gather_local_roofline(w, sp, peaks, peak_src)
     sp.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def gather_local_roofline(w, sp, peaks, peak_src, ranks=8, calls=10):
+    """The band gather of rank 0 of an emulated `ranks`-way split, on this GPU: the source ranges are token
+    ranges of the resident Q, K, V (contiguous for batch 1), the band buffers are local.  An HBM-bound copy:
+    bytes = read + write of 3 tensors x tokens x band x d x 2."""
+    import torch
+
+    import block_sparse_attention_frame_b200 as lvsa
+    from block_sparse_attention_frame_b200.sequence_parallel import head_band, token_ranges
+
+    tokens = w.T * w.P
+    n = token_ranges(tokens, ranks)
+    starts = [sum(n[:r]) for r in range(ranks)]
+    row = w.H * w.d * 2
+    tables = [[x.data_ptr() + s0 * row for s0 in starts] for x in (sp.q, sp.k, sp.v)]
+    h0, band = head_band(0, ranks, w.H)
+    bufs = [torch.empty((1, tokens, band, w.d), dtype=torch.bfloat16, device=sp.q.device) for _ in range(3)]
+    for _ in range(3):
+        lvsa.lvsa_seq_to_heads(*tables, n, h0, band, *bufs, heads=w.H)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        lvsa.lvsa_seq_to_heads(*tables, n, h0, band, *bufs, heads=w.H)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / calls
+    ok = all(torch.equal(b.view(torch.int16), x[:, :, h0:h0 + band].view(torch.int16))
+             for b, x in zip(bufs, (sp.q, sp.k, sp.v)))
+    nbytes = 2 * 3 * tokens * band * w.d * 2
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    return {"ranks_emulated": ranks, "band_heads": band, "ms": ms, "bytes": nbytes,
+            "GBps": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
+            "hbm_peak_source": f"{peak_src} copy bandwidth", "equal_to_source_heads": ok}
 
 
 def flops_per_call_dense(w) -> float:
