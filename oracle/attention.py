@@ -105,3 +105,45 @@ def dense_attention(q, k, v, scale: float | None = None) -> np.ndarray:
             out[b, :, h, :] = (E @ v[b, :, h, :]) / E.sum(axis=1, keepdims=True)
     return out
 
+
+
+def joint_token_set(t: int, lists, P: int, T: int, n_text: int) -> np.ndarray:
+    """Keys of a query token of latent frame t in a joint video + text sequence (tokens [0, T*P) are the
+    video, frame-major; [T*P, T*P + n_text) the text).  The pages only define the video part, A(t)
+    (gist.science summary, section 2 "Core Mechanism"); reading for the text (pages silent): every video
+    query also attends every text token.  A text query (t >= T) attends every token."""
+    text = np.arange(T * P, T * P + n_text, dtype=np.int64)
+    if t >= T:
+        return np.arange(0, T * P + n_text, dtype=np.int64)
+    return np.concatenate([frame_tokens(lists[int(t)], P), text])
+
+
+def joint_attention_rows(q, k, v, lists, P: int, T: int, rows, scale: float | None = None) -> np.ndarray:
+    """O for the query tokens ``rows`` of a joint sequence [batch, T*P + n_text, heads, d] (n_text taken
+    from the tensors): one softmax over joint_token_set of each row.  float64 [batch, len(rows), heads, d]."""
+    B, Ltok, H, d = q.shape
+    n_text = Ltok - T * P
+    if n_text < 0:
+        raise ValueError("tensors hold fewer than T*P tokens")
+    sigma = default_scale(d) if scale is None or scale <= 0 else float(scale)
+    rows = np.asarray(list(rows), dtype=np.int64)
+    out = np.zeros((B, rows.size, H, d), dtype=np.float64)
+    group = np.minimum(rows // P, T)  # the frame of a video row; T for every text row
+    for t in np.unique(group):
+        sel = np.nonzero(group == t)[0]
+        toks = joint_token_set(int(t), lists, P, T, n_text)
+        for b in range(B):
+            for h in range(H):
+                Q = _take(q, b, rows[sel], h)
+                K = _take(k, b, toks, h)
+                V = _take(v, b, toks, h)
+                S = sigma * (Q @ K.T)
+                m = S.max(axis=1, keepdims=True)
+                E = np.exp(S - m)
+                out[b, sel, h, :] = (E @ V) / E.sum(axis=1, keepdims=True)
+    return out
+
+
+def joint_attention(q, k, v, lists, P: int, T: int, scale: float | None = None) -> np.ndarray:
+    """O for every token of a joint video + text sequence: float64 [batch, T*P + n_text, heads, d]."""
+    return joint_attention_rows(q, k, v, lists, P, T, range(q.shape[1]), scale)
