@@ -12,7 +12,8 @@ Contents
                sets, pure integer work), plus the invariant checkers the pages
                state (budget, anchor count, rotation, coverage).
 ``attention``  softmax attention restricted to the frames of A(t), in float64
-               with numpy, and a separate plain dense attention routine.
+               with numpy, a separate plain dense attention routine, and the
+               joint video + text form (text tokens after the video).
 
 Sources (pages on "LVSA: Training-Free Sparse Attention for Long Video
 Diffusion"):
@@ -37,10 +38,15 @@ Readings where the pages are silent or disagree:
   * extension alternates right/left, right first, one new non-anchor frame per
     turn, skipping a side that reached the sequence end;
   * C >= T means every query frame attends to all T frames (dense);
-  * one joint softmax over all selected tokens, scale 1/sqrt(d) by default.
+  * one joint softmax over all selected tokens, scale 1/sqrt(d) by default;
+  * text tokens of a joint video + text sequence (pages silent; HunyuanVideo
+    1.5 is named as dual-stream in the techwalker article, section 四): every
+    video query attends them besides A(t), and a text query attends every
+    token.
 
 Parity status: every function here is pinned by tests in
-``tests/test_oracle_lists.py`` and ``tests/test_oracle_attention.py``
+``tests/test_oracle_lists.py``, ``tests/test_oracle_attention.py`` and
+``tests/test_oracle_joint.py``
 (hand-derived worked example, brute-force invariants, closed forms and a
 library masked-attention routine).  No function is "parity unpinned".
 """
