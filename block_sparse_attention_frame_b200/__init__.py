@@ -9,6 +9,7 @@ Functions carry the C ABI's names (declared in ``include/lvsa.h``):
 ``lvsa_build_frame_lists(T, C, W, step)`` -> int32 numpy array [T, min(C,T)]
 ``lvsa_build_anchors(T, C, W, step)``     -> int32 numpy array [G]
 ``lvsa_attention(q, k, v, lists, tokens_per_frame, scale=0, out=None, stream=None)``
+``lvsa_attention_joint(q, k, v, lists, tokens_per_frame, scale=0, out=None, stream=None)`` (video + text)
 ``lvsa_attention_host(q_host, k_host, v_host, lists_host, tokens_per_frame, out_host, q_dev, k_dev, v_dev,
 lists_dev, out_dev, scale=0, heads_per_band=0, stream=None)``
 ``lvsa_seq_to_heads(q_chunks, k_chunks, v_chunks, chunk_tokens, head0, band, q_band, k_band, v_band, stream=None)``
@@ -44,7 +45,7 @@ EXPORTED = [
     "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_attention_host", "lvsa_get_device_status",
     "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_exp2_fma_eval", "lvsa_status_string",
     "lvsa_version", "lvsa_seq_to_heads", "lvsa_attention_to_chunks", "lvsa_ipc_export", "lvsa_ipc_import",
-    "lvsa_ipc_release",
+    "lvsa_ipc_release", "lvsa_attention_joint",
 ]
 
 
@@ -71,6 +72,9 @@ _lib.lvsa_build_anchors.restype = _c_int
 _lib.lvsa_attention.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                 _c_float, _c_vp, _c_vp]
 _lib.lvsa_attention.restype = _c_int
+_lib.lvsa_attention_joint.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                      _c_int, _c_float, _c_vp, _c_vp]
+_lib.lvsa_attention_joint.restype = _c_int
 _lib.lvsa_attention_host.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_vp]
 _lib.lvsa_attention_host.restype = _c_int
@@ -183,6 +187,46 @@ def lvsa_attention(q, k, v, lists, tokens_per_frame: int, scale: float = 0.0, ou
                                  _stream_ptr(stream, q.device))
     _check("lvsa_attention", st)
     return out
+
+
+def lvsa_attention_joint(q, k, v, lists, tokens_per_frame: int, scale: float = 0.0, out=None, stream=None):
+    """Block-sparse attention over a joint video + text sequence.
+
+    q, k, v: CUDA bf16 [batch, T*tokens_per_frame + text_tokens, heads, d], the text tokens after the video
+    (text_tokens = the tokens beyond T*tokens_per_frame).  Video rows attend their frames' lists plus every
+    text token; text rows attend every token.  lists: CUDA int32 [T, L].  Returns ``out``.
+    """
+    import torch
+
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(x, torch.Tensor) or x.device.type != "cuda" or x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a CUDA bfloat16 tensor")
+        if not x.is_contiguous() or x.dim() != 4 or x.shape != q.shape:
+            raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q")
+    if lists.device.type != "cuda" or lists.dtype != torch.int32 or lists.dim() != 2 or not lists.is_contiguous():
+        raise TypeError("lists must be a contiguous CUDA int32 tensor [T, L]")
+    B, ntok, H, d = q.shape
+    T, L = lists.shape
+    text = ntok - T * tokens_per_frame
+    if text < 0:
+        raise ValueError(f"q has {ntok} tokens, fewer than T*tokens_per_frame = {T * tokens_per_frame}")
+    if out is None:
+        out = torch.empty_like(q)
+    elif out.shape != q.shape or out.dtype != torch.bfloat16 or not out.is_contiguous() or out.device != q.device:
+        raise ValueError("out must be a contiguous bf16 tensor shaped like q on q's device")
+    with torch.cuda.device(q.device):
+        st = _lib.lvsa_attention_joint(q.data_ptr(), k.data_ptr(), v.data_ptr(), lists.data_ptr(), L, T,
+                                       tokens_per_frame, text, H, d, B, float(scale), out.data_ptr(),
+                                       _stream_ptr(stream, q.device))
+    _check("lvsa_attention_joint", st)
+    return out
+
+
+def lvsa_attention_joint_raw(q_ptr: int, k_ptr: int, v_ptr: int, lists_ptr: int, L: int, T: int, P: int,
+                             text: int, H: int, d: int, B: int, scale: float, out_ptr: int, stream_ptr: int) -> int:
+    """The C call with raw device pointers; returns the status code unchanged."""
+    return int(_lib.lvsa_attention_joint(q_ptr, k_ptr, v_ptr, lists_ptr, L, T, P, text, H, d, B, float(scale),
+                                         out_ptr, ctypes.c_void_p(stream_ptr)))
 
 
 def lvsa_attention_raw(q_ptr: int, k_ptr: int, v_ptr: int, lists_ptr: int, L: int, T: int, P: int, H: int,

@@ -74,11 +74,11 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u
 namespace lvsa {
 namespace {
 
-// Checks shared by both attention entry points (no CUDA call).
-lvsa_status check_sizes(int L, int T, int P, int heads, int d, int batch, float scale) {
-  if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T) return LVSA_ERR_INVALID_ARG;
+// Checks shared by the attention entry points (no CUDA call).
+lvsa_status check_sizes(int L, int T, int P, int heads, int d, int batch, float scale, int text_tokens = 0) {
+  if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T || text_tokens < 0) return LVSA_ERR_INVALID_ARG;
   if (heads > 65535 || batch > 65535) return LVSA_ERR_INVALID_ARG;
-  if (static_cast<long long>(T) * P > INT_MAX) return LVSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * P + text_tokens > INT_MAX) return LVSA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return LVSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return LVSA_ERR_UNSUPPORTED;
   if (T > kMaxT) return LVSA_ERR_UNSUPPORTED;
@@ -112,20 +112,23 @@ Route one_buffer(void* out, long long tokens, int head_stride) {
 }
 
 // One launch over `heads` heads whose input rows hold `in_stride` heads; q, k, v point at the band's
-// first head.  Arguments are already validated.
+// first head.  A joint sequence holds `ntext` text tokens after the T*P video tokens.  Arguments are
+// already validated.
 lvsa_status launch_band(const void* q, const void* k, const void* v, const int32_t* lists, int L, int T, int P,
                         int heads, int in_stride, int d, int batch, float scale, const Route& route,
-                        cudaStream_t st, int dev) {
-  const int qblocks = (P + kQTiles * kBM - 1) / (kQTiles * kBM);
+                        cudaStream_t st, int dev, int ntext = 0) {
+  constexpr int kRows = kQTiles * kBM;
+  const int qblocks = (P + kRows - 1) / kRows;
   // frames of at least 256 tokens: query blocks of 256 rows run over the whole
   // sequence (a block may hold the end of one frame and the start of the next);
-  // shorter frames: blocks stay inside a frame
-  const int straddle = P >= kQTiles * kBM ? 1 : 0;
-  const long long nblocks = straddle ? (static_cast<long long>(T) * P + kQTiles * kBM - 1) / (kQTiles * kBM)
-                                     : static_cast<long long>(T) * qblocks;
+  // shorter frames: blocks stay inside a frame.  Text rows take blocks of their own.
+  const int straddle = P >= kRows ? 1 : 0;
+  const long long nvblocks = straddle ? (static_cast<long long>(T) * P + kRows - 1) / kRows
+                                      : static_cast<long long>(T) * qblocks;
+  const long long nblocks = nvblocks + (ntext + kRows - 1) / kRows;
   if (nblocks > INT_MAX) return LVSA_ERR_INVALID_ARG;
   KernelParams kp;
-  const long long tokens = static_cast<long long>(T) * P;
+  const long long tokens = static_cast<long long>(T) * P + ntext;
   if (!make_map(&kp.tm_q, q, batch, tokens, heads, in_stride, d) ||
       !make_map(&kp.tm_k, k, batch, tokens, heads, in_stride, d) ||
       !make_map(&kp.tm_v, v, batch, tokens, heads, in_stride, d))
@@ -133,6 +136,8 @@ lvsa_status launch_band(const void* q, const void* k, const void* v, const int32
   kp.lists = lists;
   kp.T = T;
   kp.P = P;
+  kp.ntext = ntext;
+  kp.nvblocks = static_cast<int>(nvblocks);
   kp.H = heads;
   kp.HS = route.head_stride;
   kp.head0 = route.head0;
@@ -206,6 +211,28 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   if (ds != LVSA_OK) return ds;
   return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale,
                      one_buffer(out, static_cast<long long>(T) * P, heads), static_cast<cudaStream_t>(stream), dev);
+}
+
+extern "C" lvsa_status lvsa_attention_joint(const void* q, const void* k, const void* v, const int32_t* lists, int L,
+                                            int T, int tokens_per_frame, int text_tokens, int heads, int d,
+                                            int batch, float scale, void* out, void* stream) {
+  using namespace lvsa;
+  const int P = tokens_per_frame;
+  if (!q || !k || !v || !lists || !out) return LVSA_ERR_INVALID_ARG;
+  if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T || text_tokens < 0) return LVSA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return LVSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lists) & 3u))
+    return LVSA_ERR_INVALID_ARG;
+  const lvsa_status cs = check_sizes(L, T, P, heads, d, batch, scale, text_tokens);
+  if (cs != LVSA_OK) return cs;
+  const long long tokens = static_cast<long long>(T) * P + text_tokens;
+  const size_t bytes = static_cast<size_t>(batch) * tokens * heads * static_cast<size_t>(d) * 2;
+  if (!disjoint(out, q, bytes) || !disjoint(out, k, bytes) || !disjoint(out, v, bytes)) return LVSA_ERR_INVALID_ARG;
+  int dev = 0;
+  const lvsa_status ds = check_device(&dev);
+  if (ds != LVSA_OK) return ds;
+  return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale, one_buffer(out, tokens, heads),
+                     static_cast<cudaStream_t>(stream), dev, text_tokens);
 }
 
 extern "C" lvsa_status lvsa_attention_to_chunks(const void* q, const void* k, const void* v, const int32_t* lists,

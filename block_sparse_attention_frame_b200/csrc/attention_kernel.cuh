@@ -83,6 +83,8 @@ struct KernelParams {
   CUtensorMap tm_v;
   const int32_t* lists;
   int T, P, H, L;    // H: heads in this launch (grid.y)
+  int ntext;         // text tokens after the T*P video tokens (joint sequence); 0: video only
+  int nvblocks;      // CTAs of video query rows per (batch, head); the text query rows take the rest
   int HS;            // heads per token row of an output buffer (H for a whole tensor, more for a band)
   int head0;         // output head of this launch's head 0 within such a row
   int nchunks;       // output rows are split by token range over nchunks buffers
@@ -153,11 +155,22 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long 
 struct FrameWalk {
   const uint32_t* ma;
   const uint32_t* mb;
-  int T, P, nwords;
+  int T, P, nwords, ntext;
   int f = 0, pos = 0, end = 0, mask = 0;
+  bool text_done = false;
 
-  __device__ FrameWalk(const uint32_t* a, const uint32_t* b_, int T_, int P_)
-      : ma(a), mb(b_), T(T_), P(P_), nwords((T_ + 31) >> 5) {}
+  __device__ FrameWalk(const uint32_t* a, const uint32_t* b_, int T_, int P_, int ntext_)
+      : ma(a), mb(b_), T(T_), P(P_), nwords((T_ + 31) >> 5), ntext(ntext_) {}
+
+  // After the frames: the text tokens of a joint sequence, one run that every query row attends.
+  __device__ __forceinline__ bool text_run() {
+    if (text_done || ntext <= 0) return false;
+    text_done = true;
+    pos = T * P;
+    end = T * P + ntext;
+    mask = 3;
+    return true;
+  }
 
   __device__ __forceinline__ int bits(int g) const {
     return static_cast<int>(((ma[g >> 5] >> (g & 31)) & 1u) | (((mb[g >> 5] >> (g & 31)) & 1u) << 1));
@@ -165,19 +178,24 @@ struct FrameWalk {
 
   __device__ __forceinline__ bool next(int& tok, int& nvalid, int& tmask) {
     while (pos >= end) {
-      if (f >= T) return false;
+      if (f >= T) {
+        if (text_run()) continue;
+        return false;
+      }
       int wi = f >> 5;
       uint32_t word = (ma[wi] | mb[wi]) & (0xffffffffu << (f & 31));
+      bool none = false;
       while (word == 0) {
         if (++wi >= nwords) {
-          f = T;
-          return false;
+          none = true;
+          break;
         }
         word = ma[wi] | mb[wi];
       }
-      const int f0 = (wi << 5) + __ffs(word) - 1;
+      const int f0 = none ? T : (wi << 5) + __ffs(word) - 1;
       if (f0 >= T) {
         f = T;
+        if (text_run()) continue;
         return false;
       }
       const int m0 = bits(f0);
@@ -319,20 +337,26 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   const int lane = threadIdx.x & 31;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
-  const int ltok = p.T * p.P;
-  // query rows [r0, r1) of the frame-major sequence: one frame fa, or fa and fb = fa + 1
+  const int vtok = p.T * p.P;      // video tokens
+  const int ltok = vtok + p.ntext;  // all tokens of a sequence
+  // query rows [r0, r1): video rows of one frame fa, or of fa and fb = fa + 1; or text rows (text_rows),
+  // which attend every frame
   int r0, r1;
-  if (p.straddle) {
-    r0 = blockIdx.x * (kQTiles * kBM);
+  const bool text_rows = blockIdx.x >= p.nvblocks;
+  if (text_rows) {
+    r0 = vtok + (blockIdx.x - p.nvblocks) * (kQTiles * kBM);
     r1 = min(r0 + kQTiles * kBM, ltok);
+  } else if (p.straddle) {
+    r0 = blockIdx.x * (kQTiles * kBM);
+    r1 = min(r0 + kQTiles * kBM, vtok);
   } else {
     const int qb = blockIdx.x % p.qblocks;
     const int t = blockIdx.x / p.qblocks;
     r0 = t * p.P + qb * (kQTiles * kBM);
     r1 = min(r0 + kQTiles * kBM, (t + 1) * p.P);
   }
-  const int fa = r0 / p.P;
-  const int fb = (r1 - 1) / p.P;
+  const int fa = text_rows ? p.T : r0 / p.P;
+  const int fb = text_rows ? p.T : (r1 - 1) / p.P;
   const bool has1 = r0 + kBM < r1;  // the second query tile has rows
   uint32_t* map_a = reinterpret_cast<uint32_t*>(smem + Cf::kOffMap);
   uint32_t* map_b = map_a + kMapWords;
@@ -340,14 +364,16 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     // frame bitmaps of the lists of fa and fb (map_b stays empty when fb == fa)
     const int nwords = (p.T + 31) >> 5;
     for (int i = threadIdx.x; i < nwords; i += kThreads) {
-      map_a[i] = 0u;
-      map_b[i] = 0u;
+      // text rows: every frame [0, T) in both maps (every run attended by every row)
+      const uint32_t all = (i < (p.T >> 5)) ? 0xffffffffu : ((1u << (p.T & 31)) - 1u);
+      map_a[i] = text_rows ? all : 0u;
+      map_b[i] = text_rows ? all : 0u;
     }
     __syncthreads();
     bool bad = false;
     const int32_t* la = p.lists + static_cast<size_t>(fa) * p.L;
     const int32_t* lb = p.lists + static_cast<size_t>(fb) * p.L;
-    const int nset = (fb != fa) ? 2 * p.L : p.L;
+    const int nset = text_rows ? 0 : (fb != fa) ? 2 * p.L : p.L;
     for (int i = threadIdx.x; i < nset; i += kThreads) {
       const int f = (i < p.L) ? __ldg(la + i) : __ldg(lb + (i - p.L));
       if (f < 0 || f >= p.T) {
@@ -429,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       ++issued;
     };
     // consumption order of the MMA warp: K0, V0, K1, V1, ...
-    FrameWalk walk(map_a, map_b, p.T, p.P);
+    FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
     int tok, nv, tmask;
     while (ok && walk.next(tok, nv, tmask)) {
       load(&p.tm_k, tok);
@@ -491,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
 
     int cidx = 0;
     bool ok = wait_all(bar_q, 0);
-    FrameWalk walk(map_a, map_b, p.T, p.P);
+    FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
     int tok, nv, tmask;
     if (ok && walk.next(tok, nv, tmask)) {
       int n_cur = (nv + 15) & ~15;
@@ -589,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       int j = 0;
       const int row = r0 + qi * kBM + r;  // query row in the frame-major sequence
       const int rbit = (row / p.P == fa) ? 1 : 2;
-      FrameWalk walk(map_a, map_b, p.T, p.P);
+      FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
       int tok, nv, tmask;
       while (walk.next(tok, nv, tmask)) {
         ok = __all_sync(0xffffffffu, wait_bounded(bar_s + qi, j & 1, w));

@@ -103,3 +103,17 @@ def make_custom(T: int, P: int, H: int, d: int, B: int = 1, seed: int = 0, devic
     w = Workload("custom", T=T, P=P, H=H, d=d, C=T, W=1, B=B, seed=seed,
                  frame_correlated_k=frame_correlated_k)
     return make_qkv(w, device=device, dtype=dtype)
+
+
+def make_joint(T: int, P: int, n_text: int, H: int, d: int, B: int = 1, seed: int = 0, device="cpu",
+               dtype=torch.bfloat16):
+    """A joint video + text sequence [batch, T*P + n_text, heads, d]: the video tokens drawn as
+    ``make_custom``, then n_text text tokens with Q, K, V ~ N(0, 1) from a generator seeded with seed + 1,
+    drawn in the order Q, K, V.  (HunyuanVideo 1.5 encodes its prompt into up to a few hundred text
+    tokens; their statistics are not available either.)"""
+    q, k, v = make_custom(T, P, H, d, B=B, seed=seed, device=device, dtype=dtype)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed + 1)
+    shape = (B, n_text, H, d)
+    tq, tk, tv = (torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(dtype) for _ in range(3))
+    return torch.cat([q, tq], dim=1), torch.cat([k, tk], dim=1), torch.cat([v, tv], dim=1)

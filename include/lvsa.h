@@ -127,6 +127,27 @@ lvsa_status lvsa_attention(const void* q, const void* k, const void* v,
                            void* out, void* stream);
 
 /*
+ * lvsa_attention_joint -- lvsa_attention over a joint video + text sequence:
+ * [batch][T*tokens_per_frame + text_tokens][heads][d], the text tokens after
+ * the frame-major video tokens (the joint attention of a dual-stream model
+ * such as HunyuanVideo 1.5, named in the techwalker article, section 四).
+ *
+ * Defines (the pages give A(t) for video frames only and say nothing of other
+ * tokens; the reading taken): a video query of frame t attends the tokens of
+ * the frames in A(t) and every text token; a text query attends every token;
+ * one softmax per row.  text_tokens = 0 is lvsa_attention exactly (the same
+ * bits).
+ *
+ * Arguments as lvsa_attention, with text_tokens >= 0 and
+ * T*tokens_per_frame + text_tokens <= INT_MAX; q, k, v, out hold the joint
+ * sequence.  Behaviour and errors as lvsa_attention.
+ */
+lvsa_status lvsa_attention_joint(const void* q, const void* k, const void* v,
+                                 const int32_t* lists, int L, int T, int tokens_per_frame,
+                                 int text_tokens, int heads, int d, int batch, float scale,
+                                 void* out, void* stream);
+
+/*
  * lvsa_attention_host -- lvsa_attention on HOST inputs and output, with the
  * transfers pipelined against the kernel by bands of heads.
  *
