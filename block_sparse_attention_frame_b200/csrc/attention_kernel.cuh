@@ -472,7 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     // Per K/V tile j:  PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): while softmax 1 works on S_1(j)
     // the tensor core runs tile 0's products, and the other way round.  Each PV is issued in two
     // halves (keys 0..63 as soon as the softmax has stored them, then keys 64..127).  The whole warp
-    // runs the schedule (descriptors stay warp-uniform); one elected lane issues.
+    // runs the schedule (descriptors stay warp-uniform); one elected lane issues each group of MMAs and
+    // the commits that follow it.  The issuer shares a sub-partition with a softmax warp of each
+    // warpgroup, so its instruction count sits on the P hand-off chain: descriptors are built as 32-bit
+    // low words, and there is one elected block per group rather than per MMA.
     const uint32_t sq = smem_u32(sQ);
     const uint32_t sr = smem_u32(sRing);
     const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
@@ -480,35 +483,29 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     const uint64_t kdesc0 = smem_desc_sw128(0, 16, 1024);
     // descriptor of an MN-major V tile: 64-wide d chunks 16 KB apart (LBO), 8-key groups 1 KB apart (SBO)
     const uint64_t vdesc0 = smem_desc_sw128(0, kChunkBytes, 1024);
+    const uint32_t khi = static_cast<uint32_t>(kdesc0 >> 32), klo0 = static_cast<uint32_t>(kdesc0);
+    const uint32_t vhi = static_cast<uint32_t>(vdesc0 >> 32), vlo0 = static_cast<uint32_t>(vdesc0);
     auto qk = [&](int i, uint32_t k_addr, int n_mma) {
-      const uint64_t qd = kdesc0 + ((sq + i * Cf::kTileBytes) >> 4);
-      const uint64_t kd = kdesc0 + (k_addr >> 4);
+      const uint32_t qd = klo0 + ((sq + i * Cf::kTileBytes) >> 4);
+      const uint32_t kd = klo0 + (k_addr >> 4);
       const uint32_t idesc = idesc_bf16_f32(kBM, n_mma, false);
-      const bool leader = elect_one();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-        if (leader) mma_ss(tmem + 128 * i, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
+        mma_ss_lo(tmem + 128 * i, qd + off, kd + off, khi, idesc, kk > 0 ? 1u : 0u);
       }
-      __syncwarp();
     };
     auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate, int k_lo, int k_hi) {
-      const uint64_t vd = vdesc0 + (v_addr >> 4);
-      const bool leader = elect_one();
+      const uint32_t vd = vlo0 + (v_addr >> 4);
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk) {
         if (kk < k_lo) continue;
         if (kk >= k_hi || kk * 16 >= n_mma) break;
-        if (leader)
-          mma_ts(tmem + kOCol0 + 128 * i, tmem + 128 * i + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
-                 (accumulate || kk > 0) ? 1u : 0u);
+        mma_ts_lo(tmem + kOCol0 + 128 * i, tmem + 128 * i + kk * 8, vd + ((kk * 16 * 128) >> 4), vhi, idesc_pv,
+                  (accumulate || kk > 0) ? 1u : 0u);
       }
-      __syncwarp();
     };
-    auto commit = [&](uint64_t* bar) {
-      if (elect_one()) mma_commit(bar);
-      __syncwarp();
-    };
+    auto commit = [&](uint64_t* bar) { mma_commit(bar); };
     auto slot_of = [&](int idx) { return idx % Cf::kSlots; };
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wait_bounded(bar, parity, w));
@@ -526,13 +523,16 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       if (ok) {
         tc_fence_after();
         const uint32_t k_addr = sr + slot_of(k0) * Cf::kTileBytes;
-        qk(0, k_addr, n_cur);
-        commit(bar_s + 0);
-        if (has1) {
-          qk(1, k_addr, n_cur);
-          commit(bar_s + 1);
+        if (elect_one()) {
+          qk(0, k_addr, n_cur);
+          commit(bar_s + 0);
+          if (has1) {
+            qk(1, k_addr, n_cur);
+            commit(bar_s + 1);
+          }
+          commit(bar_empty + slot_of(k0));
         }
-        commit(bar_empty + slot_of(k0));
+        __syncwarp();
       }
       for (int j = 0; ok; ++j) {
         int tok_n, nv_n, tmask_n;
@@ -545,7 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
           break;
         }
         tc_fence_after();
-        pv(0, v_addr, n_cur, j > 0, 0, 4);
+        if (elect_one()) pv(0, v_addr, n_cur, j > 0, 0, 4);
+        __syncwarp();
         // the next K tile is waited for while the softmax finishes P_0(j), so that nothing but the
         // P_0 hand-off stands between PV_0(j) and QK_0(j+1); commits that nobody waits on soon go
         // after the next group of MMAs
@@ -564,39 +565,51 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
           break;
         }
         tc_fence_after();
-        pv(0, v_addr, n_cur, j > 0, 4, 8);
-        if (has_next) {
-          qk(0, k_addr, n_next);
-          commit(bar_s + 0);
+        if (elect_one()) {
+          pv(0, v_addr, n_cur, j > 0, 4, 8);
+          if (has_next) {
+            qk(0, k_addr, n_next);
+            commit(bar_s + 0);
+          }
+          commit(bar_o + 0);
+          if (!has1) {
+            commit(bar_empty + slot_of(vi));
+            if (has_next) commit(bar_empty + slot_of(ki));
+          }
         }
-        commit(bar_o + 0);
+        __syncwarp();
         if (has1) {
           if (!wait_all(bar_ph + 1, j & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          pv(1, v_addr, n_cur, j > 0, 0, 4);
+          if (elect_one()) pv(1, v_addr, n_cur, j > 0, 0, 4);
+          __syncwarp();
           if (!wait_all(bar_p + 1, j & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          pv(1, v_addr, n_cur, j > 0, 4, 8);
-          if (has_next) {
-            qk(1, k_addr, n_next);
-            commit(bar_s + 1);
+          if (elect_one()) {
+            pv(1, v_addr, n_cur, j > 0, 4, 8);
+            if (has_next) {
+              qk(1, k_addr, n_next);
+              commit(bar_s + 1);
+            }
+            commit(bar_o + 1);
+            commit(bar_empty + slot_of(vi));
+            if (has_next) commit(bar_empty + slot_of(ki));
           }
-          commit(bar_o + 1);
+          __syncwarp();
         }
-        commit(bar_empty + slot_of(vi));
         if (!has_next) break;
-        commit(bar_empty + slot_of(ki));
         n_cur = n_next;
       }
     }
     // every MMA issued must be complete before TMEM is released
-    commit(bar_drain);
+    if (elect_one()) commit(bar_drain);
+    __syncwarp();
     wait_drain(bar_drain, 0, p.wait_cycles);
     __syncwarp();
   }
