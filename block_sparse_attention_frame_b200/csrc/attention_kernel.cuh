@@ -489,14 +489,15 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       const uint32_t qd = klo0 + ((sq + i * Cf::kTileBytes) >> 4);
       const uint32_t kd = klo0 + (k_addr >> 4);
       const uint32_t idesc = idesc_bf16_f32(kBM, n_mma, false);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = ((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4;
-        mma_ss_lo(tmem + 128 * i, qd + off, kd + off, khi, idesc, kk > 0 ? 1u : 0u);
-      }
+      mma_qk_group<D>(tmem + 128 * i, qd, kd, khi, idesc, 0u);
     };
     auto pv = [&](int i, uint32_t v_addr, int n_mma, bool accumulate, int k_lo, int k_hi) {
       const uint32_t vd = vlo0 + (v_addr >> 4);
+      if (n_mma >= 16 * k_hi) {  // the four 16-key steps of this half are all in the tile
+        mma_pv_group4(tmem + kOCol0 + 128 * i, tmem + 128 * i + k_lo * 8, vd + ((k_lo * 16 * 128) >> 4), vhi,
+                      idesc_pv, (accumulate || k_lo > 0) ? 1u : 0u);
+        return;
+      }
 #pragma unroll
       for (int kk = 0; kk < kBN / 16; ++kk) {
         if (kk < k_lo) continue;

@@ -143,6 +143,52 @@ __device__ __forceinline__ void mma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// A group of MMAs in one asm block: the first step takes its accumulate flag from `acc`, the others
+// accumulate.  QK^T: k-steps of 16 over a K-major SW128 operand pair, descriptor offsets (in 16-byte
+// units) (kk >> 2) * 1024 + (kk & 3) * 2.  PV: four 16-key steps, A columns + 8 and B rows + 2 KB each.
+#define LVSA_QK_STEP(OFF)                                                   \
+  "add.u32 ra, %1, " #OFF ";\n\tadd.u32 rb, %2, " #OFF ";\n\t"              \
+  "mov.b64 da, {ra, %3};\n\tmov.b64 db, {rb, %3};\n\t"                      \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pt;\n\t"
+#define LVSA_QK_HEAD                                                        \
+  "{\n\t.reg .pred pa, pt;\n\t.reg .b32 ra, rb;\n\t.reg .b64 da, db;\n\t"   \
+  "setp.ne.b32 pa, %5, 0;\n\tsetp.eq.b32 pt, %5, %5;\n\t"                   \
+  "mov.b64 da, {%1, %3};\n\tmov.b64 db, {%2, %3};\n\t"                      \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %4, pa;\n\t"
+template <int D>
+__device__ __forceinline__ void mma_qk_group(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                             uint32_t idesc, uint32_t accumulate) {
+  static_assert(D == 64 || D == 128, "head dim");
+  if constexpr (D == 128) {
+    asm volatile(LVSA_QK_HEAD LVSA_QK_STEP(2) LVSA_QK_STEP(4) LVSA_QK_STEP(6) LVSA_QK_STEP(1024)
+                     LVSA_QK_STEP(1026) LVSA_QK_STEP(1028) LVSA_QK_STEP(1030) "}" ::"r"(d_tmem),
+                 "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+                 : "memory");
+  } else {
+    asm volatile(LVSA_QK_HEAD LVSA_QK_STEP(2) LVSA_QK_STEP(4) LVSA_QK_STEP(6) "}" ::"r"(d_tmem), "r"(a_lo),
+                 "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+                 : "memory");
+  }
+}
+#define LVSA_PV_STEP(AOFF, BOFF)                                            \
+  "add.u32 ra, %1, " #AOFF ";\n\tadd.u32 rb, %2, " #BOFF ";\n\t"            \
+  "mov.b64 db, {rb, %3};\n\t"                                               \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], [ra], db, %4, pt;\n\t"
+__device__ __forceinline__ void mma_pv_group4(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred pa, pt;\n\t.reg .b32 ra, rb;\n\t.reg .b64 db;\n\t"
+      "setp.ne.b32 pa, %5, 0;\n\tsetp.eq.b32 pt, %5, %5;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, pa;\n\t"
+      LVSA_PV_STEP(8, 128) LVSA_PV_STEP(16, 256) LVSA_PV_STEP(24, 384) "}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+#undef LVSA_QK_STEP
+#undef LVSA_QK_HEAD
+#undef LVSA_PV_STEP
+
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
