@@ -186,8 +186,12 @@ def test_full_size_workloads_sampled_rows(gpu_lib, name, steps):
     w = synthetic.WORKLOADS[name]
     q, k, v = synthetic.make_qkv(w, device="cuda")
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
-    rows = sample_rows(w.T, w.P, seed=w.seed)
+    # the first step: 128 rows in each of 8 frames (frames 0, 1, T/2, T-2, T-1 and 3 seeded ones; rows 0, 1,
+    # 127, 128, the frame's last 25 and every 8th row from 1535, the rest seeded); later steps: 40 per frame
+    rows_first = sample_rows(w.T, w.P, seed=w.seed, per_frame=128)
+    rows_later = sample_rows(w.T, w.P, seed=w.seed)
     for i, s in enumerate(steps):
+        rows = rows_first if i == 0 else rows_later
         lists = gpu_lib.lvsa_build_frame_lists(w.T, w.C, w.W, s)
         out = run_kernel(gpu_lib, q, k, v, lists, w.P)
         got = out[:, rows].float().cpu().numpy()
