@@ -316,8 +316,8 @@ lvsa_status lvsa_watchdog_selftest(unsigned long long budget_ns, void* stream);
 /*
  * lvsa_exp2_fma_eval -- test hook: evaluates, element by element, the FMA-pipe
  * 2^x the attention kernel can take for a share of its softmax exponentials
- * (compiled out in this build: every exponential runs on the MUFU unit; see the
- * kernel's kPolyEvery) -- round-to-nearest range reduction plus a fitted cubic;
+ * (compiled out while the kernel's kPolyEvery is 0, as it is now: every
+ * exponential runs on the MUFU unit) -- round-to-nearest range reduction plus a fitted cubic;
  * valid for x in [-125, 126], inputs below -125 are clamped.  x, y: DEVICE float32 arrays of
  * n elements, caller-owned, 4-byte aligned; asynchronous on `stream`.
  */
