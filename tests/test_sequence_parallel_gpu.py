@@ -2,8 +2,8 @@
 attention with output rows routed to the token-range owners (lvsa_attention_to_chunks).
 
 Ranks are emulated in one process (every "peer" buffer is a local tensor; the kernels of one rank never wait
-on another's, so this is the same computation), and run for real as two processes sharing one GPU through
-CUDA IPC mappings, ordered by a gloo process group.  The outputs must equal the single call (lvsa_attention
+on another's, so this is the same computation), and run for real as two or three processes sharing one GPU
+through CUDA IPC mappings, ordered by a gloo process group.  The outputs must equal the single call (lvsa_attention
 on the whole tensors) bit for bit: every head is computed by the same kernel on the same data, only the
 buffers differ.  The single call itself is checked against the fp64 oracle in test_attention_gpu.py; the
 tiny case is checked against the oracle here too.
@@ -127,9 +127,9 @@ rank = int(os.environ["RANK"])
 dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
 torch.cuda.set_device(0)
 lvsa.lvsa_set_wait_budget_ns(500_000_000)
-T, P, H, d = 10, 300, 3, 128
+T, P, H, d = 10, 300, {heads}, 128
 q, k, v = synthetic.make_custom(T, P, H, d, seed=77, device="cuda")
-sp = SequenceParallelAttention(T, P, H, d, chunk_tokens=[1300, 1700], device="cuda:0")
+sp = SequenceParallelAttention(T, P, H, d, chunk_tokens={chunks}, device="cuda:0")
 a, b = sp.starts[rank], sp.starts[rank + 1]
 for dst, src in ((sp.q, q), (sp.k, k), (sp.v, v)):
     dst.copy_(src[:, a:b])
@@ -147,16 +147,21 @@ print("RESULT", rank, int(ok), status, flush=True)
 """
 
 
-def test_two_processes_share_one_gpu_through_ipc(tmp_path, gpu_lib):
-    """Two ranks as two processes on one GPU: each maps the other's buffers (lvsa_ipc_import), gathers its
-    heads from both, and stores its output rows into both; each rank's output equals its rows of the single
-    call.  Host barriers order the ranks; no kernel waits on the other process."""
+@pytest.mark.parametrize("world,heads,chunks", [
+    (2, 3, [1300, 1700]),
+    (3, 2, [1300, 0, 1700]),  # rank 1 holds no tokens, rank 2 no heads
+])
+def test_processes_share_one_gpu_through_ipc(tmp_path, gpu_lib, world, heads, chunks):
+    """Ranks as processes on one GPU: each maps the others' buffers (lvsa_ipc_import), gathers its heads from
+    them, and stores its output rows into them; each rank's output equals its rows of the single call.  Host
+    barriers order the ranks; no kernel waits on another process."""
     port = _free_port()
     script = tmp_path / "worker.py"
-    script.write_text(WORKER.format(root=ROOT))
+    script.write_text(WORKER.format(root=ROOT, heads=heads, chunks=chunks))
     procs = []
-    for rank in range(2):
-        env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    for rank in range(world):
+        env = dict(os.environ, RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                   MASTER_PORT=str(port))
         procs.append(subprocess.Popen([sys.executable, str(script)], env=env, stdout=subprocess.PIPE,
                                       stderr=subprocess.STDOUT, text=True))
     outs = []
