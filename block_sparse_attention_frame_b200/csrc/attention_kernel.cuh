@@ -4,7 +4,9 @@
 // section 2 "Core Mechanism" and "Complexity"): a query token of frame t attends only to the tokens of the
 // frames in A(t); one softmax over all of them; cost O(T * C * P^2 * d).
 //
-// One CTA per (256-row query block, head, batch entry); 384 threads:
+// One CTA per (256-row query block, head, batch entry); 384 threads.  In a joint video + text sequence
+// the text query rows take blocks of their own that attend every frame, and every block's walk ends with
+// one run over the text tokens (the reading taken where the pages are silent on non-video tokens).
 //   warp 8      TMA producer: both 128-row Q tiles once, then K and V tiles of the frames the block
 //               attends into a 5-slot shared-memory ring.  A block may hold the end of frame fa and the
 //               start of fa + 1; it attends the union of their lists, walked as runs of consecutive
