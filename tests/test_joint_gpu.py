@@ -29,7 +29,7 @@ def test_no_text_tokens_is_the_video_call_bit_for_bit(gpu_lib):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-@pytest.mark.parametrize("T,P,n_text,H,d,C,W,step", [
+JOINT_CASES = [
     (8, 64, 32, 2, 64, 4, 2, 3),      # the tiny shape with a short prompt
     (6, 300, 77, 3, 128, 4, 2, 1),    # straddling video blocks, one partial text tile
     (5, 256, 300, 2, 128, 3, 2, 2),   # two text blocks (256 + 44 rows), three text tiles
@@ -37,13 +37,15 @@ def test_no_text_tokens_is_the_video_call_bit_for_bit(gpu_lib):
     (9, 200, 1, 2, 128, 5, 2, 4),     # a single text token
     (3, 1560, 256, 1, 128, 2, 1, 0),  # video-sized frames
     (1, 500, 60, 2, 128, 1, 1, 0),    # T = 1: one frame and a prompt
-])
-@pytest.mark.parametrize("B", [1, 2])
+]
+
+
+# every case at batch 1, the smaller ones also at batch 2
+@pytest.mark.parametrize("T,P,n_text,H,d,C,W,step,B",
+                         [c + (1,) for c in JOINT_CASES] + [c + (2,) for c in JOINT_CASES if c[0] * c[1] <= 2000])
 def test_joint_matches_oracle(gpu_lib, T, P, n_text, H, d, C, W, step, B):
     from block_sparse_attention_frame_b200 import synthetic
 
-    if B == 2 and P * T > 2000:
-        pytest.skip("batch 2 runs on the smaller shapes only")
     q, k, v = synthetic.make_joint(T, P, n_text, H, d, B=B, seed=T + n_text, device="cpu")
     lists_np = gpu_lib.lvsa_build_frame_lists(T, C, W, step)
     out = gpu_lib.lvsa_attention_joint(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(lists_np).cuda(), P)
