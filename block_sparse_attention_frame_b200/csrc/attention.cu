@@ -275,11 +275,16 @@ extern "C" lvsa_status lvsa_attention_to_chunks(const void* q, const void* k, co
   int dev = 0;
   const lvsa_status ds = check_device(&dev);
   if (ds != LVSA_OK) return ds;
-  // a buffer in another GPU's memory (a peer mapping): its stores are released at system scope
+  // every buffer must be addressable from this GPU: its own memory, a peer mapping, or mapped (pinned)
+  // host memory, written through the device address CUDA reports for it.  A buffer that is not this
+  // GPU's memory has its stores released at system scope.
   for (int c = 0; c < nchunks; ++c) {
     if (chunk_tokens[c] == 0) continue;
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, out_chunks[c]) != cudaSuccess) return LVSA_ERR_INVALID_ARG;
+    if (at.type == cudaMemoryTypeUnregistered || at.devicePointer == nullptr) return LVSA_ERR_INVALID_ARG;
+    if (!aligned16(at.devicePointer)) return LVSA_ERR_INVALID_ARG;
+    route.out[c] = at.devicePointer;
     if (at.type != cudaMemoryTypeDevice || at.device != dev) route.routed = 1;
   }
   return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale, route, static_cast<cudaStream_t>(stream),

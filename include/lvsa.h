@@ -246,11 +246,13 @@ lvsa_status lvsa_seq_to_heads(const void* const* q_chunks, const void* const* k_
  *   q, k, v, lists, L, T, tokens_per_frame, heads, d, batch, scale  as
  *            lvsa_attention (q, k, v: [batch][T*P][heads][d], e.g. the band
  *            buffers of lvsa_seq_to_heads).
- *   out_chunks  HOST array of nchunks DEVICE pointers (this GPU's memory or a
- *            peer mapping), buffer c = [batch][chunk_tokens[c]][out_heads][d]
- *            bf16, 16-byte aligned, disjoint from q, k, v; may be NULL where
- *            chunk_tokens[c] == 0.  Heads outside [head0, head0 + heads) are
- *            not written.
+ *   out_chunks  HOST array of nchunks pointers addressable from this GPU (its
+ *            memory, a peer mapping, or pinned host memory), buffer c =
+ *            [batch][chunk_tokens[c]][out_heads][d] bf16, 16-byte aligned,
+ *            disjoint from q, k, v; may be NULL where chunk_tokens[c] == 0.
+ *            Memory CUDA does not know, or knows but cannot address from the
+ *            GPU, is refused (LVSA_ERR_INVALID_ARG).  Heads outside
+ *            [head0, head0 + heads) are not written.
  *   chunk_tokens  HOST int array, >= 0 each, summing to T * tokens_per_frame.
  *   nchunks  1..64.   out_heads, head0: head0 >= 0, head0 + heads <= out_heads.
  *   stream   a cudaStream_t (as void*).

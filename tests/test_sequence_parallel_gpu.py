@@ -189,3 +189,38 @@ def test_bench_sequence_parallel_json_line():
     assert d["scaling"] == "strong" and d["n_gpus"] == 1 and d["value"] > 0
     assert "sequence-parallel" in d["config"]["parallelism"]
     assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["gpu_launches"] == 3
+
+
+def test_rows_routed_to_host_memory_take_the_system_scope_path(gpu_lib):
+    """A range buffer that is not this GPU's memory (here pinned host memory, which the GPU addresses
+    directly) makes the kernel release its stores at system scope, the path peer stores take; the rows
+    written there equal the single call's."""
+    from block_sparse_attention_frame_b200 import synthetic
+
+    T, P, H, d = 6, 300, 2, 128
+    q, k, v = synthetic.make_custom(T, P, H, d, seed=13, device="cuda")
+    lists = torch.from_numpy(gpu_lib.lvsa_build_frame_lists(T, 4, 2, 3)).cuda()
+    ref = gpu_lib.lvsa_attention(q, k, v, lists, P)
+    chunks = [1000, 800]
+    dev_part = torch.full((1, chunks[0], H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    host_part = torch.full((1, chunks[1], H, d), float("nan"), dtype=torch.bfloat16).pin_memory()
+    gpu_lib.lvsa_attention_to_chunks(q, k, v, lists, P, [dev_part, host_part.data_ptr()], chunks, H, 0)
+    torch.cuda.synchronize()
+    assert gpu_lib.lvsa_get_device_status(clear=True) == 0
+    assert same_bits(dev_part, ref[:, :chunks[0]])
+    assert same_bits(host_part, ref[:, chunks[0]:].cpu())
+
+
+def test_unaddressable_range_buffer_is_refused(gpu_lib):
+    """Pageable host memory cannot be written by the GPU: the call returns an argument error before any
+    launch."""
+    from block_sparse_attention_frame_b200 import synthetic
+
+    T, P, H, d = 4, 256, 1, 128
+    q, k, v = synthetic.make_custom(T, P, H, d, seed=3, device="cuda")
+    lists = torch.from_numpy(gpu_lib.lvsa_build_frame_lists(T, 3, 1, 0)).cuda()
+    dev_part = torch.empty((1, 512, H, d), dtype=torch.bfloat16, device="cuda")
+    pageable = torch.empty((1, 512, H, d), dtype=torch.bfloat16)  # not pinned
+    with pytest.raises(gpu_lib.LvsaError) as e:
+        gpu_lib.lvsa_attention_to_chunks(q, k, v, lists, P, [dev_part, pageable.data_ptr()], [512, 512], H, 0)
+    assert e.value.status == gpu_lib.LVSA_ERR_INVALID_ARG
