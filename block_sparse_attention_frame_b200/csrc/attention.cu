@@ -48,7 +48,7 @@ std::mutex g_attr_mu;
 bool g_attr_set[2][64] = {};
 
 template <int D>
-lvsa_status launch(const KernelParams& kp, int B, cudaStream_t stream, int dev) {
+lvsa_status launch(const KernelParams& kp, int nlaunch, int B, cudaStream_t stream, int dev) {
   using Cf = Cfg<D>;
   const int di = (D == 128) ? 1 : 0;
   {
@@ -61,7 +61,7 @@ lvsa_status launch(const KernelParams& kp, int B, cudaStream_t stream, int dev) 
       g_attr_set[di][dev] = true;
     }
   }
-  dim3 grid(static_cast<unsigned>(kp.nblocks), static_cast<unsigned>(kp.H), static_cast<unsigned>(B));
+  dim3 grid(static_cast<unsigned>(nlaunch), static_cast<unsigned>(kp.H), static_cast<unsigned>(B));
   lvsa_attention_kernel<D><<<grid, kThreads, Cf::kSmemBytes, stream>>>(kp);
   return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
 }
@@ -111,22 +111,40 @@ Route one_buffer(void* out, long long tokens, int head_stride) {
   return r;
 }
 
+// Query blocks of a launch over T*P video tokens and ntext text tokens (256-row blocks over the whole
+// sequence when frames hold at least 256 tokens, else blocks inside each frame; text rows after them).
+struct Blocks {
+  int straddle, qblocks;
+  long long nvblocks, nblocks;
+};
+Blocks query_blocks(int T, int P, int ntext) {
+  constexpr int kRows = kQTiles * kBM;
+  Blocks bl;
+  bl.qblocks = (P + kRows - 1) / kRows;
+  bl.straddle = P >= kRows ? 1 : 0;
+  bl.nvblocks = bl.straddle ? (static_cast<long long>(T) * P + kRows - 1) / kRows : static_cast<long long>(T) * bl.qblocks;
+  bl.nblocks = bl.nvblocks + (ntext + kRows - 1) / kRows;
+  return bl;
+}
+
 // One launch over `heads` heads whose input rows hold `in_stride` heads; q, k, v point at the band's
-// first head.  A joint sequence holds `ntext` text tokens after the T*P video tokens.  Arguments are
-// already validated.
+// first head.  A joint sequence holds `ntext` text tokens after the T*P video tokens.  The launch covers
+// query blocks [block0, block0 + nlaunch) (nlaunch < 0: every block).  Arguments are already validated.
 lvsa_status launch_band(const void* q, const void* k, const void* v, const int32_t* lists, int L, int T, int P,
                         int heads, int in_stride, int d, int batch, float scale, const Route& route,
-                        cudaStream_t st, int dev, int ntext = 0) {
-  constexpr int kRows = kQTiles * kBM;
-  const int qblocks = (P + kRows - 1) / kRows;
+                        cudaStream_t st, int dev, int ntext = 0, int block0 = 0, int nlaunch = -1) {
   // frames of at least 256 tokens: query blocks of 256 rows run over the whole
   // sequence (a block may hold the end of one frame and the start of the next);
   // shorter frames: blocks stay inside a frame.  Text rows take blocks of their own.
-  const int straddle = P >= kRows ? 1 : 0;
-  const long long nvblocks = straddle ? (static_cast<long long>(T) * P + kRows - 1) / kRows
-                                      : static_cast<long long>(T) * qblocks;
-  const long long nblocks = nvblocks + (ntext + kRows - 1) / kRows;
+  const Blocks bl = query_blocks(T, P, ntext);
+  const int qblocks = bl.qblocks, straddle = bl.straddle;
+  const long long nvblocks = bl.nvblocks, nblocks = bl.nblocks;
   if (nblocks > INT_MAX) return LVSA_ERR_INVALID_ARG;
+  if (nlaunch < 0) {
+    block0 = 0;
+    nlaunch = static_cast<int>(nblocks);
+  }
+  if (block0 < 0 || nlaunch < 1 || block0 + static_cast<long long>(nlaunch) > nblocks) return LVSA_ERR_INVALID_ARG;
   KernelParams kp;
   const long long tokens = static_cast<long long>(T) * P + ntext;
   if (!make_map(&kp.tm_q, q, batch, tokens, heads, in_stride, d) ||
@@ -150,10 +168,11 @@ lvsa_status launch_band(const void* q, const void* k, const void* v, const int32
   kp.qblocks = qblocks;
   kp.straddle = straddle;
   kp.nblocks = static_cast<int>(nblocks);
+  kp.block0 = block0;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   kp.scale_log2 = sc * 1.4426950408889634f;
   kp.wait_cycles = static_cast<long long>(static_cast<double>(g_wait_ns) * kBudgetCyclesPerNs);
-  return d == 128 ? launch<128>(kp, batch, st, dev) : launch<64>(kp, batch, st, dev);
+  return d == 128 ? launch<128>(kp, nlaunch, batch, st, dev) : launch<64>(kp, nlaunch, batch, st, dev);
 }
 
 // Streams and events of the host-buffer path, created once per device and kept: one upload and one
@@ -161,7 +180,7 @@ lvsa_status launch_band(const void* q, const void* k, const void* v, const int32
 // SMs the previous band's last wave leaves free.
 struct HostPipe {
   cudaStream_t h2d = nullptr, d2h = nullptr, k[2] = {nullptr, nullptr};
-  std::vector<cudaEvent_t> ev;  // 2 per band + 2
+  std::vector<cudaEvent_t> ev;  // 2 per launch (a band, or a piece of one) + 2
 };
 std::mutex g_pipe_mu;
 HostPipe g_pipe[64];
@@ -173,7 +192,7 @@ lvsa_status pipe_for(int dev, int bands, HostPipe** out) {
   if (!hp.d2h && cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess) return LVSA_ERR_CUDA;
   for (int i = 0; i < 2; ++i)
     if (!hp.k[i] && cudaStreamCreateWithFlags(&hp.k[i], cudaStreamNonBlocking) != cudaSuccess) return LVSA_ERR_CUDA;
-  const size_t need = 2 * static_cast<size_t>(bands) + 2;
+  const size_t need = 2 * static_cast<size_t>(bands) + 2;  // `bands`: launches the call may make
   while (hp.ev.size() < need) {
     cudaEvent_t e;
     if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return LVSA_ERR_CUDA;
@@ -322,12 +341,21 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
   // video sizes (T*P/256 query blocks per batch entry)
   const int hb = heads_per_band > 0 ? heads_per_band : 1;
   const int bands = (heads + hb - 1) / hb;
+  // The first band's Q is uploaded, and the last band's output read back, in pieces of whole query blocks,
+  // each piece's kernel launched (or its rows read back) as soon as it can: only a quarter of a band's Q
+  // upload precedes the first kernel, and only a quarter of a band's readback follows the last one.
+  // (Batch 1 and frames of at least 256 tokens, where a piece of query blocks is one range of rows.)
+  constexpr int kPieces = 4;
+  const Blocks bl = query_blocks(T, P, 0);
+  const bool pieces = batch == 1 && bl.straddle && bl.nvblocks >= 2 * kPieces;
   std::lock_guard<std::mutex> g(g_pipe_mu);
   HostPipe* hp = nullptr;
-  lvsa_status r = pipe_for(dev, bands, &hp);
+  lvsa_status r = pipe_for(dev, bands + 2 * kPieces, &hp);  // at most 2 bands go in pieces
   if (r != LVSA_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaEvent_t ev_start = hp->ev[2 * bands], ev_done = hp->ev[2 * bands + 1];
+  int next_ev = 0;
+  auto event = [&]() { return hp->ev[next_ev++]; };
+  cudaEvent_t ev_start = event(), ev_done = event();
   auto ok = [](cudaError_t e) { return e == cudaSuccess; };
   // the copies into the staging buffers wait for earlier work on the caller's stream
   if (!ok(cudaEventRecord(ev_start, st)) || !ok(cudaStreamWaitEvent(hp->h2d, ev_start, 0)) ||
@@ -338,24 +366,48 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
   const char* src[3] = {static_cast<const char*>(q_host), static_cast<const char*>(k_host),
                         static_cast<const char*>(v_host)};
   char* dst[3] = {static_cast<char*>(q_dev), static_cast<char*>(k_dev), static_cast<char*>(v_dev)};
+  const long long tokens = static_cast<long long>(T) * P;
+  constexpr int kRows = kQTiles * kBM;
   for (int gi = 0; gi < bands; ++gi) {
     const int h0 = gi * hb;
     const int hn = std::min(hb, heads - h0);
     const size_t off = static_cast<size_t>(h0) * d * 2;
     const size_t width = static_cast<size_t>(hn) * d * 2;
-    cudaEvent_t ev_in = hp->ev[2 * gi], ev_k = hp->ev[2 * gi + 1];
-    // band gi of Q, K, V: a column band of every token row
-    for (int t = 0; t < 3; ++t)
+    const bool q_in_pieces = pieces && gi == 0;
+    const bool out_in_pieces = pieces && gi == bands - 1;
+    const int npieces = (q_in_pieces || out_in_pieces) ? kPieces : 1;
+    // band gi of K, V (and Q, unless it goes up in pieces): a column band of every token row
+    for (int t = q_in_pieces ? 1 : 0; t < 3; ++t)
       if (!ok(cudaMemcpy2DAsync(dst[t] + off, row_bytes, src[t] + off, row_bytes, width, rows, cudaMemcpyHostToDevice,
                                 hp->h2d)))
         return LVSA_ERR_CUDA;
-    cudaStream_t ks = hp->k[gi & 1];
-    if (!ok(cudaEventRecord(ev_in, hp->h2d)) || !ok(cudaStreamWaitEvent(ks, ev_in, 0))) return LVSA_ERR_CUDA;
-    r = launch_band(dst[0] + off, dst[1] + off, dst[2] + off, lists_dev, L, T, P, hn, heads, d, batch, scale,
-                    one_buffer(static_cast<char*>(out_dev) + off, static_cast<long long>(T) * P, heads), ks, dev);
-    if (r != LVSA_OK) return r;
-    if (!ok(cudaEventRecord(ev_k, ks)) || !ok(cudaStreamWaitEvent(hp->d2h, ev_k, 0))) return LVSA_ERR_CUDA;
-    if (!ok(cudaMemcpy2DAsync(static_cast<char*>(out_host) + off, row_bytes, static_cast<const char*>(out_dev) + off,
+    for (int c = 0; c < npieces; ++c) {
+      // query blocks [b0, b1) = rows [b0 * 256, b1 * 256) of the sequence
+      const long long b0 = npieces == 1 ? 0 : bl.nvblocks * c / npieces;
+      const long long b1 = npieces == 1 ? bl.nvblocks : bl.nvblocks * (c + 1) / npieces;
+      const size_t row0 = static_cast<size_t>(b0) * kRows;
+      const size_t nrows = static_cast<size_t>(std::min(b1 * kRows, tokens)) - row0;
+      if (q_in_pieces &&
+          !ok(cudaMemcpy2DAsync(dst[0] + row0 * row_bytes + off, row_bytes, src[0] + row0 * row_bytes + off, row_bytes,
+                                width, nrows, cudaMemcpyHostToDevice, hp->h2d)))
+        return LVSA_ERR_CUDA;
+      cudaEvent_t ev_in = event(), ev_k = event();
+      cudaStream_t ks = hp->k[(gi + c) & 1];
+      if (!ok(cudaEventRecord(ev_in, hp->h2d)) || !ok(cudaStreamWaitEvent(ks, ev_in, 0))) return LVSA_ERR_CUDA;
+      r = launch_band(dst[0] + off, dst[1] + off, dst[2] + off, lists_dev, L, T, P, hn, heads, d, batch, scale,
+                      one_buffer(static_cast<char*>(out_dev) + off, tokens, heads), ks, dev, 0,
+                      npieces == 1 ? 0 : static_cast<int>(b0), npieces == 1 ? -1 : static_cast<int>(b1 - b0));
+      if (r != LVSA_OK) return r;
+      if (!ok(cudaEventRecord(ev_k, ks)) || !ok(cudaStreamWaitEvent(hp->d2h, ev_k, 0))) return LVSA_ERR_CUDA;
+      if (out_in_pieces &&
+          !ok(cudaMemcpy2DAsync(static_cast<char*>(out_host) + row0 * row_bytes + off, row_bytes,
+                                static_cast<const char*>(out_dev) + row0 * row_bytes + off, row_bytes, width, nrows,
+                                cudaMemcpyDeviceToHost, hp->d2h)))
+        return LVSA_ERR_CUDA;
+    }
+    // the whole band's output, once every piece's kernel is done
+    if (!out_in_pieces &&
+        !ok(cudaMemcpy2DAsync(static_cast<char*>(out_host) + off, row_bytes, static_cast<const char*>(out_dev) + off,
                               row_bytes, width, rows, cudaMemcpyDeviceToHost, hp->d2h)))
       return LVSA_ERR_CUDA;
   }

@@ -95,7 +95,8 @@ struct KernelParams {
   __nv_bfloat16* out_chunk[kMaxChunks];      // of every batch entry: [batch][tokens of c][HS][d]
   int straddle;      // 1: CTA c takes query rows [256c, 256c+256) of the whole frame-major sequence
   int qblocks;       // straddle == 0: ceil(P / 256) CTAs per query frame
-  int nblocks;       // CTAs per (batch, head)
+  int nblocks;       // query blocks per (batch, head)
+  int block0;        // query block of blockIdx.x == 0 (a launch may cover a range of the blocks)
   float scale_log2;  // softmax scale * log2(e)
   long long wait_cycles;
 };
@@ -344,16 +345,17 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   // query rows [r0, r1): video rows of one frame fa, or of fa and fb = fa + 1; or text rows (text_rows),
   // which attend every frame
   int r0, r1;
-  const bool text_rows = blockIdx.x >= p.nvblocks;
+  const int qblk = blockIdx.x + p.block0;  // this CTA's query block
+  const bool text_rows = qblk >= p.nvblocks;
   if (text_rows) {
-    r0 = vtok + (blockIdx.x - p.nvblocks) * (kQTiles * kBM);
+    r0 = vtok + (qblk - p.nvblocks) * (kQTiles * kBM);
     r1 = min(r0 + kQTiles * kBM, ltok);
   } else if (p.straddle) {
-    r0 = blockIdx.x * (kQTiles * kBM);
+    r0 = qblk * (kQTiles * kBM);
     r1 = min(r0 + kQTiles * kBM, vtok);
   } else {
-    const int qb = blockIdx.x % p.qblocks;
-    const int t = blockIdx.x / p.qblocks;
+    const int qb = qblk % p.qblocks;
+    const int t = qblk / p.qblocks;
     r0 = t * p.P + qb * (kQTiles * kBM);
     r1 = min(r0 + kQTiles * kBM, (t + 1) * p.P);
   }

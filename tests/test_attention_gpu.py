@@ -271,6 +271,10 @@ def run_host_path(lib, q, k, v, lists_np, P, heads_per_band=0, scale=0.0):
     (8, 64, 2, 64, 1, 4, 2, 1, 0),      # automatic bands
     (6, 300, 3, 128, 2, 3, 1, 4, 2),    # straddling query blocks, batch 2, uneven bands (2 + 1 heads)
     (5, 96, 5, 64, 1, 5, 2, 0, 3),      # dense lists, ragged frames, bands of 3 + 2
+    # batch 1, 256-row blocks: the first band's Q goes up, and the last band's output comes back, in pieces
+    (10, 300, 3, 128, 1, 5, 2, 3, 1),   # three bands: first and last in pieces
+    (10, 300, 2, 128, 1, 5, 2, 3, 1),   # two bands
+    (10, 300, 3, 128, 1, 5, 2, 3, 3),   # one band, both in pieces
 ])
 def test_host_buffer_path_equals_device_path(gpu_lib, T, P, H, d, B, C, W, s, hb):
     q, k, v = make(T, P, H, d, B=B, seed=11)
