@@ -176,3 +176,24 @@ def test_ipc_calls_reject_null_and_unknown_pointers(lib):
     assert lib._lib.lvsa_ipc_release(ctypes.c_void_p(1 << 24)) == lib.LVSA_ERR_INVALID_ARG  # never imported
     with pytest.raises(ValueError):
         lib.lvsa_ipc_import(b"short")
+
+
+def test_attention_joint_argument_validation_without_gpu(lib):
+    A, M = 1 << 24, 1 << 20
+    good = dict(q=A, k=A + M, v=A + 2 * M, lists=A + 3 * M, L=4, T=8, P=64, text=32, H=2, d=64, B=1, scale=0.0,
+                out=A + 4 * M)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return lib.lvsa_attention_joint_raw(a["q"], a["k"], a["v"], a["lists"], a["L"], a["T"], a["P"], a["text"],
+                                            a["H"], a["d"], a["B"], a["scale"], a["out"], 0)
+
+    INV = lib.LVSA_ERR_INVALID_ARG
+    assert call(text=-1) == INV
+    assert call(T=2, P=1 << 30, text=1 << 30) == INV   # video + text tokens past INT_MAX
+    assert call(out=A + 2 * M + 16) == INV               # output overlaps v
+    assert call(q=0) == INV
+    assert call(L=9) == INV
+    assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
+    assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
+    assert call(text=0) in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
