@@ -191,7 +191,6 @@ def test_attention_joint_argument_validation_without_gpu(lib):
     INV = lib.LVSA_ERR_INVALID_ARG
     assert call(text=-1) == INV
     assert call(T=1, L=1, P=1 << 30, text=1 << 30) == INV  # video tokens fit, video + text pass INT_MAX
-    assert call(T=1, L=1, P=1 << 30, text=0) != INV
     assert call(out=A + 2 * M + 16) == INV               # output overlaps v
     assert call(q=0) == INV
     assert call(L=9) == INV
