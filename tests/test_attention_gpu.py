@@ -165,7 +165,9 @@ def test_watchdog_times_out_and_context_survives(gpu_lib):
 def sample_rows(T, P, seed, per_frame=40):
     g = np.random.default_rng(seed)
     frames = sorted(set([0, 1, T // 2, T - 2, T - 1] + list(g.choice(T, 3, replace=False))))
-    base = sorted(set([0, 1, 127, 128, P - 25, P - 24, P - 1] + list(range(min(1535, P - 1), P, 8))))
+    # rows 0, 1, 127, 128 and the last 25 rows of the frame (its 24-row tail past the last full 128-row
+    # tile at P = 1560, and the row before it)
+    base = sorted(set([0, 1, 127, 128] + list(range(max(0, P - 25), P))))
     rows = []
     for f in frames:
         extra = g.choice(P, max(0, per_frame - len(base)), replace=False)
@@ -187,7 +189,7 @@ def test_full_size_workloads_sampled_rows(gpu_lib, name, steps):
     q, k, v = synthetic.make_qkv(w, device="cuda")
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     # the first step: 128 rows in each of 8 frames (frames 0, 1, T/2, T-2, T-1 and 3 seeded ones; rows 0, 1,
-    # 127, 128, the frame's last 25 and every 8th row from 1535, the rest seeded); later steps: 40 per frame
+    # 127, 128 and the frame's last 25, the rest seeded); later steps: 40 per frame
     rows_first = sample_rows(w.T, w.P, seed=w.seed, per_frame=128)
     rows_later = sample_rows(w.T, w.P, seed=w.seed)
     for i, s in enumerate(steps):
