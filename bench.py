@@ -156,13 +156,17 @@ def barrier(world: int):
         dist.barrier()
 
 
+ORACLE_KIND = ("oracle: fp64 numpy, one (head, query frame) at a time; its matrix products run in numpy's BLAS "
+               "dgemm on `cores` threads")
+
+
 def cpu_oracle_sample(w, seconds: float, seed: int = 0):
     """Time the fp64 oracle on whole (head, query-frame) units of the workload
     until ``seconds`` of CPU work are done.  Returns (flops, elapsed, units)."""
     import numpy as np
     import torch
 
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
     from oracle import attention as OA
     from oracle import lists as OL
 
@@ -187,6 +191,7 @@ def cpu_oracle_sample(w, seconds: float, seed: int = 0):
 
 
 def host_threads() -> int:
+    """Threads the oracle's matrix products run on (numpy's BLAS pool)."""
     try:
         import threadpoolctl
 
@@ -197,9 +202,61 @@ def host_threads() -> int:
         return os.cpu_count() or 1
 
 
+def host_info() -> dict:
+    """The host the CPU legs ran on: logical CPUs available to this process and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except Exception:
+        pass
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except Exception:
+        nproc = os.cpu_count()
+    return {"nproc": nproc, "cpu_model": model, "blas_threads": host_threads()}
+
+
+# The pages' own figures, quoted as context only (another machine, end-to-end or host-side; no kernel timing):
+# techwalker article "华为巴黎研究院让AI视频“不再原地打转”", sections 二, 三 and 四.
+PAGES_CONTEXT = {
+    "end_to_end_generation_single_80GB_gpu": [
+        {"model": "Wan 2.1 1.3B", "frames": 481, "dense_min": 51, "lvsa_min": 16, "speedup": 3.17},
+        {"model": "Wan 2.1 14B", "frames": 481, "dense_min": 238, "lvsa_min": 80, "speedup": 2.98},
+        {"model": "HunyuanVideo 1.5", "frames": 193, "dense_min": 80, "lvsa_min": 24, "speedup": 3.33},
+    ],
+    "host_window_extension": "about 1.4 us per frame, at most 200 us per step (section 二)",
+    "host_anchor_recompute": "under 1 ms for the longest 121-frame sequence (section 三)",
+    "source": "techwalker article, sections 二, 三, 四; context only, not a target",
+}
+
+# The list configurations of the five workloads (T, C, W), timed for the oracle's list build.
+LIST_CONFIGS = {"tiny": (8, 4, 2), "wan1.3b_1x": (21, 21, 9), "wan1.3b_6x": (121, 21, 9), "wan14b_6x": (121, 21, 9),
+                "hunyuan1.5_1.5x": (49, 33, 13)}
+
+
+def oracle_list_build_us(steps: int = 50) -> dict:
+    """The oracle's frame-list build (Python sets, by definition) timed per step over steps 0..steps-1 for
+    the list configuration of every workload: median and max microseconds per step."""
+    from oracle import lists as OL
+
+    res = {}
+    for name, (T, C, W) in LIST_CONFIGS.items():
+        us = []
+        for s in range(steps):
+            t0 = time.perf_counter()
+            OL.frame_lists(T, C, W, s)
+            us.append((time.perf_counter() - t0) * 1e6)
+        res[name] = {"T": T, "C": C, "W": W, "median_us": statistics.median(us), "max_us": max(us)}
+    return res
+
+
 def run_reference(args, rank, world):
     """The oracle as it stands, on the host cores: each step one bounded sample."""
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     if rank != 0:
         return 0
@@ -216,17 +273,43 @@ def run_reference(args, rank, world):
     value = tot_f / tot_t / 1e12
     ms_call = flops_per_call(w) / (value * 1e12) * 1e3
     sample = (f"{units} (head, query frame) units of {w.P} query rows each over {args.steps} steps "
-              f"(~{per_step:.1f} s per step), extrapolated to the full call")
+              f"(~{per_step:.1f} s per step); value = sampled FLOPs / sampled time")
+    info = host_info()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_call, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "full_call_ms_extrapolated": ms_call, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": workload_config(w, world),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": info["blas_threads"], "kind": ORACLE_KIND,
+                         "sample": sample, "nproc": info["nproc"], "cpu_model": info["cpu_model"]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_cpu_full_calls(args, rank):
+    """The oracle's whole call, timed on the host cores, for the two workloads small enough to finish in
+    minutes: the tiny case (step 3) and Wan-1.3B at its 1x horizon (C = T: dense).  One JSON line."""
+    import synthetic
+    from oracle import attention as OA
+    from oracle import lists as OL
+
+    if rank != 0:
+        return 0
+    res = []
+    for name, step in (("tiny", 3), ("wan1.3b_1x", 0)):
+        w = synthetic.WORKLOADS[name]
+        q, k, v = synthetic.make_qkv(w, device="cpu")
+        t0 = time.perf_counter()
+        lists = OL.frame_lists(w.T, w.C, w.W, step)
+        OA.sparse_attention(q, k, v, lists, w.P)
+        t = time.perf_counter() - t0
+        res.append({"workload": name, "step": step, "seconds": t, "tflops": flops_per_call(w) / t / 1e12})
+    info = host_info()
+    print(json.dumps({"oracle_full_calls": res, "cores": info["blas_threads"], "nproc": info["nproc"],
+                      "cpu_model": info["cpu_model"], "kind": ORACLE_KIND}), flush=True)
     return 0
 
 
@@ -246,11 +329,11 @@ def workload_config(w, world, fixed_grid=False):
 
 
 def run_lvsa(args, rank, world, local):
-    import numpy as np
     import torch
 
     import block_sparse_attention_frame_b200 as lvsa
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
+    from block_sparse_attention_frame_b200.pipeline import StepPipeline, host_lists
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -271,28 +354,14 @@ def run_lvsa(args, rank, world, local):
     calls = 1 if shard else world    # per step, over all ranks: sharded ranks share one call
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream(dev)
-    nsteps = args.warmup + args.steps
-    # per-step pinned host list buffers (the host writes step s+1 while step s copies)
-    pinned = [torch.empty((w.T, w.L), dtype=torch.int32).pin_memory() for _ in range(nsteps)]
-    lists_dev = torch.empty((w.T, w.L), dtype=torch.int32, device=dev)
-    build_us = []
-
-    def list_step(s):
-        # fixed-grid ablation: the anchors never rotate, i.e. the step-0 pattern at every step
-        return 0 if args.fixed_grid else s
-
-    def step(s, host_list_buf):
-        t0 = time.perf_counter()
-        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, list_step(s), out=host_list_buf.numpy())
-        build_us.append((time.perf_counter() - t0) * 1e6)
-        lists_dev.copy_(host_list_buf, non_blocking=True)
-        lvsa.lvsa_attention(q, k, v, lists_dev, w.P, out=out, stream=stream)
+    # the per-step path: host list build into a pinned ring buffer, async upload, kernel
+    pipe = StepPipeline(w.T, w.C, w.W, w.P, dev, fixed_grid=args.fixed_grid)
 
     # ---------------------------------------------------------------- device-resident timing
     for s in range(args.warmup):
-        step(s, pinned[s])
+        pipe.step(s, q, k, v, out, stream)
     torch.cuda.synchronize()
-    build_us.clear()
+    pipe.build_us.clear()
     ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -300,19 +369,13 @@ def run_lvsa(args, rank, world, local):
     with ClockSampler(local) as clocks:
         start.record(stream)
         for i in range(args.steps):
-            s = args.warmup + i
-            t0 = time.perf_counter()
-            lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, list_step(s), out=pinned[s].numpy())
-            build_us.append((time.perf_counter() - t0) * 1e6)
-            lists_dev.copy_(pinned[s], non_blocking=True)
-            ev_k[i][0].record(stream)
-            lvsa.lvsa_attention(q, k, v, lists_dev, w.P, out=out, stream=stream)
-            ev_k[i][1].record(stream)
+            pipe.step(args.warmup + i, q, k, v, out, stream, kernel_events=ev_k[i])
         stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = max_over_ranks(start.elapsed_time(stop), world)
     kernel_ms = [a.elapsed_time(b) for a, b in ev_k]
+    build_us = list(pipe.build_us)
     status = lvsa.lvsa_get_device_status(clear=True)
     if status:
         raise RuntimeError(f"device status {status:#x} after the timed region")
@@ -325,18 +388,26 @@ def run_lvsa(args, rank, world, local):
         return 0
 
     # ---------------------------------------------------------------- dense control (same kernel, C = T)
+    # step by step: the sparse call of step s, then the same kernel with every frame listed
     dense_lists = torch.from_numpy(lvsa.lvsa_build_frame_lists(w.T, w.T, 1, 0)).to(dev)
     dout = torch.empty_like(q)
     lvsa.lvsa_attention(q, k, v, dense_lists, w.P, out=dout)
     torch.cuda.synchronize()
-    dense_calls = 2
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    d0.record(stream)
-    for _ in range(dense_calls):
-        lvsa.lvsa_attention(q, k, v, dense_lists, w.P, out=dout)
-    d1.record(stream)
-    torch.cuda.synchronize()
-    dense_ms = d0.elapsed_time(d1) / dense_calls
+    ncmp = args.dense_compare_steps
+    if ncmp < 0:
+        ncmp = args.steps if w.name.startswith("hunyuan") else min(3, args.steps)
+    per_step = []
+    for i in range(ncmp):
+        s = args.warmup + i
+        es, ed = ((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2))
+        pipe.step(s, q, k, v, out, stream, kernel_events=es)
+        ed[0].record(stream)
+        lvsa.lvsa_attention(q, k, v, dense_lists, w.P, out=dout, stream=stream)
+        ed[1].record(stream)
+        torch.cuda.synchronize()
+        sp, dn = es[0].elapsed_time(es[1]), ed[0].elapsed_time(ed[1])
+        per_step.append({"step": s, "sparse_ms": sp, "dense_ms": dn, "speedup": dn / sp})
+    dense_ms = statistics.mean(x["dense_ms"] for x in per_step)
     del dout
 
     # ---------------------------------------------------------------- end to end with host buffers
@@ -345,21 +416,28 @@ def run_lvsa(args, rank, world, local):
     vh = v.cpu().pin_memory()
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     e2e_steps = max(3, min(args.steps, 10))
+    # one pinned host list buffer per end-to-end step: the call copies it asynchronously
+    e2e_lists = [torch.empty((w.T, w.L), dtype=torch.int32).pin_memory() for _ in range(e2e_steps + 1)]
+    lists_dev = torch.empty((w.T, w.L), dtype=torch.int32, device=dev)
 
-    def e2e_step(s):
+    def e2e_step(i, s):
         # the public host-buffer call: uploads of Q, K, V, the list and the readback of O are
         # inside it, pipelined against the kernel by bands of heads
-        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, list_step(s), out=pinned[s % nsteps].numpy())
-        lvsa.lvsa_attention_host(qh, kh, vh, pinned[s % nsteps], w.P, oh, q, k, v, lists_dev, out,
+        torch.cuda.nvtx.range_push("lvsa.build_lists")
+        host_lists(w.T, w.C, w.W, s, args.fixed_grid, out=e2e_lists[i].numpy())
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.nvtx.range_push("lvsa.attention_host")
+        lvsa.lvsa_attention_host(qh, kh, vh, e2e_lists[i], w.P, oh, q, k, v, lists_dev, out,
                                  heads_per_band=args.heads_per_band, stream=stream)
+        torch.cuda.nvtx.range_pop()
 
-    e2e_step(0)
+    e2e_step(e2e_steps, 0)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(e2e_steps):
-        e2e_step(i)
+        e2e_step(i, args.warmup + i)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
@@ -405,15 +483,21 @@ def run_lvsa(args, rank, world, local):
                         f"{args.heads_per_band or 1} head(s))"},
         "gpu_launches": args.steps,
         "dense_control": {"ms_per_call": dense_ms, "tflops": flops_per_call_dense(w) / (dense_ms * 1e-3) / 1e12,
-                          "speedup_sparse_vs_dense": dense_ms / kern_avg_ms},
-        "list_build_us": {"median": statistics.median(build_us), "max": max(build_us)},
+                          "speedup_sparse_vs_dense": statistics.mean(x["speedup"] for x in per_step),
+                          "per_step": per_step},
+        "list_build_us": {"median": statistics.median(build_us), "max": max(build_us),
+                          "what": "lvsa_build_frame_lists (C ABI) into the pinned ring buffer, per timed step"},
         "clocks": clocks.summary(),
+        "pages_context": PAGES_CONTEXT,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, t, units = cpu_oracle_sample(w, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": host_threads(), "kind": "oracle",
+        info = host_info()
+        line["cpu_baseline"] = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": info["blas_threads"],
+                                "kind": ORACLE_KIND, "nproc": info["nproc"], "cpu_model": info["cpu_model"],
                                 "sample": f"{units} (head, query frame) units of {w.P} rows, "
-                                          f"{t:.1f} s of fp64 numpy on the host"}
+                                          f"{t:.1f} s of fp64 numpy on the host",
+                                "list_build_us_per_step": oracle_list_build_us()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -425,7 +509,7 @@ def run_sweep(args, rank, world, local):
     import torch
 
     import block_sparse_attention_frame_b200 as lvsa
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     if rank != 0:
         return 0
@@ -468,7 +552,7 @@ def run_sequence_parallel(args, rank, world, local):
     import torch
 
     import block_sparse_attention_frame_b200 as lvsa
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
     from block_sparse_attention_frame_b200.sequence_parallel import SequenceParallelAttention
 
     dev = torch.device("cuda", local)
@@ -651,6 +735,12 @@ def main(argv=None):
                          "instead of running a replica per rank")
     ap.add_argument("--sequence-parallel", action="store_true",
                     help="split one call over the ranks by token ranges (Ulysses layout, peer-memory exchanges)")
+    ap.add_argument("--dense-compare-steps", type=int, default=-1,
+                    help="steps timed sparse then dense (C = T) one after the other (-1: every timed step for "
+                         "the HunyuanVideo workloads, 3 otherwise)")
+    ap.add_argument("--cpu-full-calls", action="store_true",
+                    help="time the oracle's full call on the tiny and Wan-1.3B 1x workloads (minutes of CPU) "
+                         "and print one JSON line")
     ap.add_argument("--heads-per-band", type=int, default=0,
                     help="end-to-end call: heads per pipelined band (0: one)")
     args = ap.parse_args(argv)
@@ -659,6 +749,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             return run_reference(args, rank, world)
+        if args.cpu_full_calls:
+            return run_cpu_full_calls(args, rank)
         if args.sweep:
             return run_sweep(args, rank, world, local)
         if args.sequence_parallel:

@@ -43,7 +43,7 @@ LVSA_IPC_HANDLE_BYTES = 72
 
 EXPORTED = [
     "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_attention_host", "lvsa_get_device_status",
-    "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_exp2_fma_eval", "lvsa_status_string",
+    "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_status_string",
     "lvsa_version", "lvsa_seq_to_heads", "lvsa_attention_to_chunks", "lvsa_ipc_export", "lvsa_ipc_import",
     "lvsa_ipc_release", "lvsa_attention_joint",
 ]
@@ -96,8 +96,6 @@ _lib.lvsa_set_wait_budget_ns.argtypes = [_c_ull]
 _lib.lvsa_set_wait_budget_ns.restype = _c_int
 _lib.lvsa_watchdog_selftest.argtypes = [_c_ull, _c_vp]
 _lib.lvsa_watchdog_selftest.restype = _c_int
-_lib.lvsa_exp2_fma_eval.argtypes = [_c_vp, _c_vp, _c_int, _c_vp]
-_lib.lvsa_exp2_fma_eval.restype = _c_int
 _lib.lvsa_status_string.argtypes = [_c_int]
 _lib.lvsa_status_string.restype = ctypes.c_char_p
 _lib.lvsa_version.argtypes = []
@@ -148,6 +146,13 @@ def lvsa_build_anchors(T: int, C: int, W: int, step: int) -> np.ndarray:
     return out
 
 
+def _same_device(q, **others):
+    """Every tensor of a call on q's GPU: the kernel addresses them from that device."""
+    for name, x in others.items():
+        if x.device != q.device:
+            raise ValueError(f"{name} is on {x.device}, q on {q.device}: every tensor of a call must be on one GPU")
+
+
 def _stream_ptr(stream, device):
     import torch
 
@@ -173,6 +178,7 @@ def lvsa_attention(q, k, v, lists, tokens_per_frame: int, scale: float = 0.0, ou
             raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q")
     if lists.device.type != "cuda" or lists.dtype != torch.int32 or lists.dim() != 2 or not lists.is_contiguous():
         raise TypeError("lists must be a contiguous CUDA int32 tensor [T, L]")
+    _same_device(q, k=k, v=v, lists=lists)
     B, ntok, H, d = q.shape
     T, L = lists.shape
     if ntok != T * tokens_per_frame:
@@ -205,6 +211,7 @@ def lvsa_attention_joint(q, k, v, lists, tokens_per_frame: int, scale: float = 0
             raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q")
     if lists.device.type != "cuda" or lists.dtype != torch.int32 or lists.dim() != 2 or not lists.is_contiguous():
         raise TypeError("lists must be a contiguous CUDA int32 tensor [T, L]")
+    _same_device(q, k=k, v=v, lists=lists)
     B, ntok, H, d = q.shape
     T, L = lists.shape
     text = ntok - T * tokens_per_frame
@@ -356,6 +363,7 @@ def lvsa_attention_to_chunks(q, k, v, lists, tokens_per_frame: int, out_chunks, 
             raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q")
     if lists.device.type != "cuda" or lists.dtype != torch.int32 or lists.dim() != 2 or not lists.is_contiguous():
         raise TypeError("lists must be a contiguous CUDA int32 tensor [T, L]")
+    _same_device(q, k=k, v=v, lists=lists)
     if len(out_chunks) != len(chunk_tokens):
         raise ValueError("one token count per output buffer")
     for x, n in zip(out_chunks, chunk_tokens):
@@ -363,6 +371,9 @@ def lvsa_attention_to_chunks(q, k, v, lists, tokens_per_frame: int, out_chunks, 
                                             or x.shape[1:] != (n, out_heads, q.shape[3])):
             raise ValueError("an output buffer tensor must be contiguous bf16 [batch, tokens of its range, "
                              "out_heads, d]")
+        if isinstance(x, torch.Tensor) and x.device != q.device:
+            raise ValueError("an output buffer tensor must be on q's GPU; another GPU's buffer is passed as the "
+                             "address lvsa_ipc_import returned")
     B, ntok, H, d = q.shape
     T, L = lists.shape
     if ntok != T * tokens_per_frame:
@@ -411,15 +422,3 @@ def lvsa_watchdog_selftest(budget_ns: int, stream=None) -> None:
     _check("lvsa_watchdog_selftest",
            _lib.lvsa_watchdog_selftest(int(budget_ns), _stream_ptr(stream, torch.cuda.current_device())))
 
-
-def lvsa_exp2_fma_eval(x, stream=None):
-    """The kernel's FMA-pipe 2^x on a CUDA float32 tensor (test hook)."""
-    import torch
-
-    if x.device.type != "cuda" or x.dtype != torch.float32 or not x.is_contiguous():
-        raise TypeError("x must be a contiguous CUDA float32 tensor")
-    y = torch.empty_like(x)
-    with torch.cuda.device(x.device):
-        _check("lvsa_exp2_fma_eval",
-               _lib.lvsa_exp2_fma_eval(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream, x.device)))
-    return y

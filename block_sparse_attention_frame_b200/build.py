@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "liblvsa.so")
 
 SOURCES = ["lists.cpp", "attention.cu", "exchange.cu"]
-HEADERS = [os.path.join(INCLUDE, "lvsa.h"), os.path.join(CSRC, "sm100.cuh"), os.path.join(CSRC, "attention_kernel.cuh")]
+HEADERS = [os.path.join(INCLUDE, "lvsa.h"), os.path.join(CSRC, "sm100.cuh"), os.path.join(CSRC, "attention_kernel.cuh"),
+           os.path.join(CSRC, "buffer_checks.h")]
 
 
 def nvcc_path() -> str:

@@ -1,12 +1,16 @@
 // Host side of the LVSA attention path: tensor maps, launches and the C ABI entry points
 // lvsa_attention (device buffers) and lvsa_attention_host (host buffers, transfers pipelined by bands of
 // heads), plus the status and test hooks declared in lvsa.h.  The kernel is in attention_kernel.cuh.
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <climits>
+#include <cstdio>
 #include <mutex>
 #include <vector>
 
 #include "attention_kernel.cuh"
+#include "buffer_checks.h"
 
 namespace lvsa {
 // ------------------------------------------------------------------ host side
@@ -171,7 +175,7 @@ lvsa_status launch_band(const void* q, const void* k, const void* v, const int32
   kp.block0 = block0;
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   kp.scale_log2 = sc * 1.4426950408889634f;
-  kp.wait_cycles = static_cast<long long>(static_cast<double>(g_wait_ns) * kBudgetCyclesPerNs);
+  kp.wait_cycles = wait_budget_cycles(g_wait_ns);
   return d == 128 ? launch<128>(kp, nlaunch, batch, st, dev) : launch<64>(kp, nlaunch, batch, st, dev);
 }
 
@@ -202,10 +206,23 @@ lvsa_status pipe_for(int dev, int bands, HostPipe** out) {
   return LVSA_OK;
 }
 
-bool disjoint(const void* a, const void* b, size_t bytes) {
-  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x + bytes <= y || y + bytes <= x;
-}
+bool disjoint(const void* a, const void* b, size_t bytes) { return ranges_disjoint(a, bytes, b, bytes); }
+
+// A named range on a profiler's host timeline (NVTX).  With no profiler attached a push or pop is a call
+// that returns at once.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  NvtxRange(const char* what, int band) {
+    char buf[48];
+    std::snprintf(buf, sizeof(buf), "%s %d", what, band);
+    nvtxRangePushA(buf);
+  }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+PeerOps runtime_peer_ops() { return PeerOps{cudaDeviceCanAccessPeer, cudaDeviceEnablePeerAccess, cudaGetLastError}; }
 
 }  // namespace
 }  // namespace lvsa
@@ -225,6 +242,7 @@ extern "C" lvsa_status lvsa_attention(const void* q, const void* k, const void* 
   if (cs != LVSA_OK) return cs;
   const size_t bytes = static_cast<size_t>(batch) * T * P * heads * static_cast<size_t>(d) * 2;
   if (!disjoint(out, q, bytes) || !disjoint(out, k, bytes) || !disjoint(out, v, bytes)) return LVSA_ERR_INVALID_ARG;
+  if (!ranges_disjoint(out, bytes, lists, static_cast<size_t>(T) * L * 4)) return LVSA_ERR_INVALID_ARG;
   int dev = 0;
   const lvsa_status ds = check_device(&dev);
   if (ds != LVSA_OK) return ds;
@@ -247,6 +265,7 @@ extern "C" lvsa_status lvsa_attention_joint(const void* q, const void* k, const 
   const long long tokens = static_cast<long long>(T) * P + text_tokens;
   const size_t bytes = static_cast<size_t>(batch) * tokens * heads * static_cast<size_t>(d) * 2;
   if (!disjoint(out, q, bytes) || !disjoint(out, k, bytes) || !disjoint(out, v, bytes)) return LVSA_ERR_INVALID_ARG;
+  if (!ranges_disjoint(out, bytes, lists, static_cast<size_t>(T) * L * 4)) return LVSA_ERR_INVALID_ARG;
   int dev = 0;
   const lvsa_status ds = check_device(&dev);
   if (ds != LVSA_OK) return ds;
@@ -273,39 +292,58 @@ extern "C" lvsa_status lvsa_attention_to_chunks(const void* q, const void* k, co
   route.head_stride = out_heads;
   route.head0 = head0;
   long long tokens = 0;
-  const size_t in_bytes = static_cast<size_t>(batch) * T * P * heads * static_cast<size_t>(d) * 2;
   for (int c = 0; c < nchunks; ++c) {
     if (chunk_tokens[c] < 0) return LVSA_ERR_INVALID_ARG;
     route.start[c] = static_cast<int>(tokens);
     tokens += chunk_tokens[c];
     if (tokens > static_cast<long long>(T) * P) return LVSA_ERR_INVALID_ARG;
     route.out[c] = out_chunks[c];
-    if (chunk_tokens[c] == 0) continue;
-    if (!out_chunks[c] || !aligned16(out_chunks[c])) return LVSA_ERR_INVALID_ARG;
-    const size_t cb = static_cast<size_t>(batch) * chunk_tokens[c] * out_heads * static_cast<size_t>(d) * 2;
-    const uintptr_t o = reinterpret_cast<uintptr_t>(out_chunks[c]);
-    for (const void* in : {q, k, v}) {
-      const uintptr_t x = reinterpret_cast<uintptr_t>(in);
-      if (!(o + cb <= x || x + in_bytes <= o)) return LVSA_ERR_INVALID_ARG;
-    }
+    if (chunk_tokens[c] > 0 && (!out_chunks[c] || !aligned16(out_chunks[c]))) return LVSA_ERR_INVALID_ARG;
   }
   if (tokens != static_cast<long long>(T) * P) return LVSA_ERR_INVALID_ARG;
   route.start[nchunks] = static_cast<int>(tokens);
+  // output buffers disjoint from each other, from q, k, v and from the lists: checked on the caller's
+  // addresses here (no CUDA call), and again below on the device addresses CUDA reports for them
+  auto overlaps = [&](void* const* outs) {
+    const size_t in_bytes = static_cast<size_t>(batch) * T * P * heads * static_cast<size_t>(d) * 2;
+    const size_t list_bytes = static_cast<size_t>(T) * L * 4;
+    for (int c = 0; c < nchunks; ++c) {
+      if (chunk_tokens[c] == 0) continue;
+      const size_t cb = static_cast<size_t>(batch) * chunk_tokens[c] * out_heads * static_cast<size_t>(d) * 2;
+      for (const void* in : {q, k, v})
+        if (!ranges_disjoint(outs[c], cb, in, in_bytes)) return true;
+      if (!ranges_disjoint(outs[c], cb, lists, list_bytes)) return true;
+      for (int e = 0; e < c; ++e) {
+        const size_t eb = static_cast<size_t>(batch) * chunk_tokens[e] * out_heads * static_cast<size_t>(d) * 2;
+        if (!ranges_disjoint(outs[c], cb, outs[e], eb)) return true;
+      }
+    }
+    return false;
+  };
+  if (overlaps(out_chunks)) return LVSA_ERR_INVALID_ARG;
   int dev = 0;
   const lvsa_status ds = check_device(&dev);
   if (ds != LVSA_OK) return ds;
-  // every buffer must be addressable from this GPU: its own memory, a peer mapping, or mapped (pinned)
-  // host memory, written through the device address CUDA reports for it.  A buffer that is not this
-  // GPU's memory has its stores released at system scope.
+  // every buffer must be addressable from this GPU: its own memory, another GPU's with peer access, or
+  // mapped (pinned) host memory, written through the device address CUDA reports for it.  A buffer that is
+  // not this GPU's memory has its stores released at system scope.
+  const PeerOps ops = runtime_peer_ops();
   for (int c = 0; c < nchunks; ++c) {
     if (chunk_tokens[c] == 0) continue;
     cudaPointerAttributes at;
-    if (cudaPointerGetAttributes(&at, out_chunks[c]) != cudaSuccess) return LVSA_ERR_INVALID_ARG;
-    if (at.type == cudaMemoryTypeUnregistered || at.devicePointer == nullptr) return LVSA_ERR_INVALID_ARG;
-    if (!aligned16(at.devicePointer)) return LVSA_ERR_INVALID_ARG;
-    route.out[c] = at.devicePointer;
-    if (at.type != cudaMemoryTypeDevice || at.device != dev) route.routed = 1;
+    if (cudaPointerGetAttributes(&at, out_chunks[c]) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return LVSA_ERR_INVALID_ARG;
+    }
+    void* dptr = nullptr;
+    int remote = 0;
+    const lvsa_status as = device_address(at, dev, ops, &dptr, &remote);
+    if (as != LVSA_OK) return as;
+    if (!aligned16(dptr)) return LVSA_ERR_INVALID_ARG;
+    route.out[c] = dptr;
+    route.routed |= remote;
   }
+  if (overlaps(route.out)) return LVSA_ERR_INVALID_ARG;
   return launch_band(q, k, v, lists, L, T, P, heads, heads, d, batch, scale, route, static_cast<cudaStream_t>(stream),
                      dev);
 }
@@ -333,6 +371,9 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
     return LVSA_ERR_INVALID_ARG;
   if (!disjoint(out_host, q_host, bytes) || !disjoint(out_host, k_host, bytes) || !disjoint(out_host, v_host, bytes))
     return LVSA_ERR_INVALID_ARG;
+  const size_t list_bytes = static_cast<size_t>(T) * L * 4;
+  if (!ranges_disjoint(out_dev, bytes, lists_dev, list_bytes) || !ranges_disjoint(out_host, bytes, lists_host, list_bytes))
+    return LVSA_ERR_INVALID_ARG;
   int dev = 0;
   const lvsa_status ds = check_device(&dev);
   if (ds != LVSA_OK) return ds;
@@ -349,6 +390,7 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
   const Blocks bl = query_blocks(T, P, 0);
   const bool pieces = batch == 1 && bl.straddle && bl.nvblocks >= 2 * kPieces;
   std::lock_guard<std::mutex> g(g_pipe_mu);
+  NvtxRange whole("lvsa_attention_host");
   HostPipe* hp = nullptr;
   lvsa_status r = pipe_for(dev, bands + 2 * kPieces, &hp);  // at most 2 bands go in pieces
   if (r != LVSA_OK) return r;
@@ -377,10 +419,13 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
     const bool out_in_pieces = pieces && gi == bands - 1;
     const int npieces = (q_in_pieces || out_in_pieces) ? kPieces : 1;
     // band gi of K, V (and Q, unless it goes up in pieces): a column band of every token row
-    for (int t = q_in_pieces ? 1 : 0; t < 3; ++t)
-      if (!ok(cudaMemcpy2DAsync(dst[t] + off, row_bytes, src[t] + off, row_bytes, width, rows, cudaMemcpyHostToDevice,
-                                hp->h2d)))
-        return LVSA_ERR_CUDA;
+    {
+      NvtxRange r("lvsa.upload band", gi);
+      for (int t = q_in_pieces ? 1 : 0; t < 3; ++t)
+        if (!ok(cudaMemcpy2DAsync(dst[t] + off, row_bytes, src[t] + off, row_bytes, width, rows,
+                                  cudaMemcpyHostToDevice, hp->h2d)))
+          return LVSA_ERR_CUDA;
+    }
     for (int c = 0; c < npieces; ++c) {
       // query blocks [b0, b1) = rows [b0 * 256, b1 * 256) of the sequence
       const long long b0 = npieces == 1 ? 0 : bl.nvblocks * c / npieces;
@@ -391,6 +436,7 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
           !ok(cudaMemcpy2DAsync(dst[0] + row0 * row_bytes + off, row_bytes, src[0] + row0 * row_bytes + off, row_bytes,
                                 width, nrows, cudaMemcpyHostToDevice, hp->h2d)))
         return LVSA_ERR_CUDA;
+      NvtxRange kr("lvsa.kernel band", gi);
       cudaEvent_t ev_in = event(), ev_k = event();
       cudaStream_t ks = hp->k[(gi + c) & 1];
       if (!ok(cudaEventRecord(ev_in, hp->h2d)) || !ok(cudaStreamWaitEvent(ks, ev_in, 0))) return LVSA_ERR_CUDA;
@@ -406,6 +452,7 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
         return LVSA_ERR_CUDA;
     }
     // the whole band's output, once every piece's kernel is done
+    NvtxRange rr("lvsa.readback band", gi);
     if (!out_in_pieces &&
         !ok(cudaMemcpy2DAsync(static_cast<char*>(out_host) + off, row_bytes, static_cast<const char*>(out_dev) + off,
                               row_bytes, width, rows, cudaMemcpyDeviceToHost, hp->d2h)))
@@ -431,24 +478,15 @@ extern "C" lvsa_status lvsa_get_device_status(unsigned int* flags, int clear) {
 }
 
 extern "C" lvsa_status lvsa_set_wait_budget_ns(unsigned long long ns) {
-  lvsa::g_wait_ns = ns < 1000ull ? 1000ull : ns;
+  if (ns > lvsa::kMaxWaitBudgetNs) return LVSA_ERR_INVALID_ARG;
+  lvsa::g_wait_ns = ns < lvsa::kMinWaitBudgetNs ? lvsa::kMinWaitBudgetNs : ns;
   return LVSA_OK;
 }
 
 extern "C" lvsa_status lvsa_watchdog_selftest(unsigned long long budget_ns, void* stream) {
   if (budget_ns < 1000ull) budget_ns = 1000ull;
   if (budget_ns > 10000000000ull) return LVSA_ERR_INVALID_ARG;
-  lvsa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<long long>(static_cast<double>(budget_ns) * lvsa::kBudgetCyclesPerNs));
-  return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
-}
-
-extern "C" lvsa_status lvsa_exp2_fma_eval(const float* x, float* y, int n, void* stream) {
-  if (!x || !y || n < 0 || (reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u))
-    return LVSA_ERR_INVALID_ARG;
-  if (n == 0) return LVSA_OK;
-  const int pairs = (n + 1) / 2;
-  lvsa::exp2_fma_eval_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  lvsa::watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(lvsa::wait_budget_cycles(budget_ns));
   return cudaGetLastError() == cudaSuccess ? LVSA_OK : LVSA_ERR_CUDA;
 }
 

@@ -22,6 +22,7 @@
 #include <map>
 #include <mutex>
 
+#include "buffer_checks.h"
 #include "lvsa.h"
 
 namespace lvsa {
@@ -74,10 +75,7 @@ __global__ void __launch_bounds__(kGatherThreads) seq_to_heads_kernel(const __gr
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
-bool disjoint(const void* a, size_t abytes, const void* b, size_t bbytes) {
-  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-  return x + abytes <= y || y + bbytes <= x;
-}
+bool disjoint(const void* a, size_t abytes, const void* b, size_t bbytes) { return ranges_disjoint(a, abytes, b, bbytes); }
 
 // ------------------------------------------------------------------ IPC mappings
 using AddrRangeFn = CUresult (*)(CUdeviceptr*, size_t*, CUdeviceptr);
@@ -162,6 +160,25 @@ extern "C" lvsa_status lvsa_seq_to_heads(const void* const* q_chunks, const void
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LVSA_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LVSA_ERR_CUDA;
+  // every source range must be addressable from this GPU (its memory, a peer's with peer access, or mapped
+  // host memory); the kernel loads through the device address CUDA reports for it
+  const PeerOps ops{cudaDeviceCanAccessPeer, cudaDeviceEnablePeerAccess, cudaGetLastError};
+  for (int c = 0; c < nchunks; ++c) {
+    if (chunk_tokens[c] == 0) continue;
+    for (int x = 0; x < 3; ++x) {
+      cudaPointerAttributes at;
+      if (cudaPointerGetAttributes(&at, tables[x][c]) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return LVSA_ERR_INVALID_ARG;
+      }
+      void* dptr = nullptr;
+      int remote = 0;
+      const lvsa_status as = device_address(at, dev, ops, &dptr, &remote);
+      if (as != LVSA_OK) return as;
+      if (!aligned16(dptr)) return LVSA_ERR_INVALID_ARG;
+      gp.src[x][c] = static_cast<const uint4*>(dptr);
+    }
+  }
   const int vx = gp.vec_band < kGatherThreads ? gp.vec_band : kGatherThreads;
   const int ry = kGatherThreads / vx;
   // about 8 CTAs of 256 threads per SM over the whole launch, at least one per source range

@@ -258,29 +258,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA pipe for x in [-125, 126]: x = j + f with j = round(x) taken from the
-// low mantissa bits of x + 1.5*2^23, f in [-1/2, 1/2]; 2^f by a cubic fitted here to the
-// relative error (csrc/fit_exp2_poly.py: max relative error 7.5e-5 in float32 Horner
-// form); the exponent j is added to the bit pattern of the cubic's value.
-constexpr float kExp2C0 = 0x1.fff694p-1f;
-constexpr float kExp2C1 = 0x1.62f31ap-1f;
-constexpr float kExp2C2 = 0x1.f0ddf6p-3f;
-constexpr float kExp2C3 = 0x1.c3f6f0p-5f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
-  const float2 t = fadd2(x, make_float2(kRoundMagic, kRoundMagic));
-  const float2 j = fadd2(t, make_float2(-kRoundMagic, -kRoundMagic));
-  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);
-  float2 p = ffma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
-  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
 // Two floats -> packed bf16x2 (round to nearest even); `lo` lands in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

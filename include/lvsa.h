@@ -111,7 +111,7 @@ lvsa_status lvsa_build_anchors(int T, int C, int W, long long step,
  *            T <= 4096 (LVSA_ERR_UNSUPPORTED above).
  *   scale    softmax scale; <= 0 selects 1/sqrt(d).
  *   out      DEVICE bf16, same layout as q, 16-byte aligned, must not overlap
- *            q, k or v.
+ *            q, k, v or lists.
  *   stream   a cudaStream_t (passed as void*), NULL = default stream.
  * Behaviour: asynchronous on `stream`; returns after the launch.  Argument and
  * launch errors are returned here.  A device-side wait that runs out (a hung
@@ -164,10 +164,11 @@ lvsa_status lvsa_attention_joint(const void* q, const void* k, const void* v,
  *            Page-locked (pinned) memory is needed for the copies to overlap.
  *   lists_host  HOST int32 [T][L] (as written by lvsa_build_frame_lists).
  *   L, T, tokens_per_frame, heads, d, batch, scale  as lvsa_attention.
- *   out_host HOST bf16, same layout as q_host; must not overlap q/k/v_host.
+ *   out_host HOST bf16, same layout as q_host; must not overlap q/k/v_host or
+ *            lists_host.
  *   q_dev, k_dev, v_dev, out_dev  DEVICE staging buffers of the full tensor
  *            size (batch*T*tokens_per_frame*heads*d bf16 each), caller-owned,
- *            16-byte aligned; out_dev must not overlap q/k/v_dev.  On return
+ *            16-byte aligned; out_dev must not overlap q/k/v_dev or lists_dev.  On return
  *            from the stream they hold the inputs and the output.
  *   lists_dev   DEVICE int32 [T][L] staging buffer, 4-byte aligned.
  *   heads_per_band  heads per band, 1..heads; 0 = one head per band.
@@ -214,10 +215,13 @@ lvsa_status lvsa_attention_host(const void* q_host, const void* k_host, const vo
  * bit).
  *
  * Arguments:
- *   q_chunks, k_chunks, v_chunks  HOST arrays of nchunks DEVICE pointers (this
- *            GPU's memory or a peer mapping), chunk c = [batch][chunk_tokens[c]]
- *            [heads][d] bf16, 16-byte aligned; may be NULL where
- *            chunk_tokens[c] == 0.
+ *   q_chunks, k_chunks, v_chunks  HOST arrays of nchunks pointers this GPU can
+ *            address (its memory, another GPU's with peer access -- enabled
+ *            here if it is not yet -- or a peer mapping, or pinned host memory),
+ *            chunk c = [batch][chunk_tokens[c]][heads][d] bf16, 16-byte aligned;
+ *            may be NULL where chunk_tokens[c] == 0.  A pointer the GPU cannot
+ *            address (pageable host memory, another GPU without peer access) is
+ *            refused with LVSA_ERR_INVALID_ARG before any launch.
  *   chunk_tokens  HOST int array of nchunks token counts (>= 0, sum >= 1);
  *            ranges follow one another in array order.
  *   nchunks  1..64.   heads, head0, band: 0 <= head0, 1 <= band,
@@ -247,12 +251,14 @@ lvsa_status lvsa_seq_to_heads(const void* const* q_chunks, const void* const* k_
  *            lvsa_attention (q, k, v: [batch][T*P][heads][d], e.g. the band
  *            buffers of lvsa_seq_to_heads).
  *   out_chunks  HOST array of nchunks pointers addressable from this GPU (its
- *            memory, a peer mapping, or pinned host memory), buffer c =
+ *            memory, another GPU's with peer access -- enabled here if it is
+ *            not yet -- a peer mapping, or pinned host memory), buffer c =
  *            [batch][chunk_tokens[c]][out_heads][d] bf16, 16-byte aligned,
- *            disjoint from q, k, v; may be NULL where chunk_tokens[c] == 0.
- *            Memory CUDA does not know, or knows but cannot address from the
- *            GPU, is refused (LVSA_ERR_INVALID_ARG).  Heads outside
- *            [head0, head0 + heads) are not written.
+ *            disjoint from each other, from q, k, v and from lists; may be NULL
+ *            where chunk_tokens[c] == 0.  Memory CUDA does not know, or knows
+ *            but cannot address from the GPU (pageable host memory, another
+ *            GPU without peer access), is refused (LVSA_ERR_INVALID_ARG).
+ *            Heads outside [head0, head0 + heads) are not written.
  *   chunk_tokens  HOST int array, >= 0 each, summing to T * tokens_per_frame.
  *   nchunks  1..64.   out_heads, head0: head0 >= 0, head0 + heads <= out_heads.
  *   stream   a cudaStream_t (as void*).
@@ -303,7 +309,9 @@ lvsa_status lvsa_get_device_status(unsigned int* flags, int clear);
 
 /*
  * lvsa_set_wait_budget_ns -- time budget of every device-side wait of later
- * launches (default 4e9 ns).  Values below 1000 ns are raised to 1000 ns.
+ * launches (default 4e9 ns, counted in SM cycles at 2 cycles per ns).  Values
+ * below 1000 ns are raised to 1000 ns; values above 1e12 ns (1000 s) are
+ * refused with LVSA_ERR_INVALID_ARG and the budget is left unchanged.
  */
 lvsa_status lvsa_set_wait_budget_ns(unsigned long long ns);
 
@@ -314,16 +322,6 @@ lvsa_status lvsa_set_wait_budget_ns(unsigned long long ns);
  * kernel returns normally (no trap, no fault).  Used to test failure detection.
  */
 lvsa_status lvsa_watchdog_selftest(unsigned long long budget_ns, void* stream);
-
-/*
- * lvsa_exp2_fma_eval -- test hook: evaluates, element by element, the FMA-pipe
- * 2^x the attention kernel can take for a share of its softmax exponentials
- * (compiled out while the kernel's kPolyEvery is 0, as it is now: every
- * exponential runs on the MUFU unit) -- round-to-nearest range reduction plus a fitted cubic;
- * valid for x in [-125, 126], inputs below -125 are clamped.  x, y: DEVICE float32 arrays of
- * n elements, caller-owned, 4-byte aligned; asynchronous on `stream`.
- */
-lvsa_status lvsa_exp2_fma_eval(const float* x, float* y, int n, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* lvsa_status_string(int status);

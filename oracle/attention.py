@@ -24,22 +24,30 @@ import math
 import numpy as np
 
 
+def _host_tensor(x):
+    """A torch tensor given to the oracle must already be in host memory: the oracle never touches a GPU."""
+    if x.device.type != "cpu":
+        raise ValueError(f"the oracle takes host tensors only (got one on {x.device}); pass x.cpu()")
+    return x
+
+
 def _f64(x) -> np.ndarray:
-    if hasattr(x, "detach"):  # torch tensor -> numpy (CPU), any float dtype
+    if hasattr(x, "detach"):  # torch tensor (host memory, any float dtype) -> float64 numpy
         import torch
 
-        x = x.detach().to("cpu").to(torch.float64).numpy()
+        x = _host_tensor(x).detach().to(torch.float64).numpy()
     return np.asarray(x, dtype=np.float64)
 
 
 def _take(x, b: int, tokens: np.ndarray, h: int) -> np.ndarray:
-    """x[b, tokens, h, :] as float64 (gathered before widening, so a large
-    bf16 torch tensor is never converted whole)."""
+    """x[b, tokens, h, :] as float64.  A torch tensor (host memory) is gathered
+    before it is widened, so a large bf16 tensor is never converted whole; the
+    widening bf16/fp32 -> float64 is exact either way."""
     if hasattr(x, "detach"):
         import torch
 
-        idx = torch.as_tensor(tokens, dtype=torch.long, device=x.device)
-        return x[b].index_select(0, idx)[:, h, :].detach().to("cpu").to(torch.float64).numpy()
+        idx = torch.as_tensor(tokens, dtype=torch.long)
+        return _host_tensor(x)[b].index_select(0, idx)[:, h, :].detach().to(torch.float64).numpy()
     return np.asarray(x[b, tokens, h, :], dtype=np.float64)
 
 

@@ -64,6 +64,7 @@ def test_attention_argument_validation_without_gpu(lib):
     assert call(out=A + 64) == INV       # overlaps q (and k, v) without being equal
     assert call(q=A + 8) == INV          # not 16-byte aligned
     assert call(lists=A + 3 * M + 2) == INV  # int32 misaligned
+    assert call(lists=A + 4 * M + 256) == INV  # the output overlaps the device lists
     assert call(scale=float("nan")) == INV
     assert call(T=1 << 20, P=1 << 12) == INV  # T*P overflows int32
     assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
@@ -99,6 +100,8 @@ def test_host_path_argument_validation_without_gpu(lib):
     assert call(lists_dev=A + 11 * n + 2) == INV  # int32 misaligned
     assert call(out_dev=A + 8 * n + 64) == INV    # output staging overlaps q_dev
     assert call(out_host=A + n // 2) == INV       # host output overlaps q_host
+    assert call(lists_dev=A + 12 * n + 64) == INV  # output staging overlaps the device lists
+    assert call(lists_host=A + 4 * n + 64) == INV  # host output overlaps the host lists
     assert call(L=0) == INV and call(T=0) == INV
     assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
     from conftest import cuda_available
@@ -156,6 +159,9 @@ def test_attention_to_chunks_argument_validation_without_gpu(lib):
     assert call(outs=[A + 4 * M, 0, A + 6 * M]) != INV  # an empty range does not
     assert call(outs=[A + 4 * M + 8, A + 5 * M, A + 6 * M]) == INV
     assert call(outs=[A + 4 * M, A + 5 * M, A + 2 * M]) == INV  # an output buffer overlaps v
+    assert call(outs=[A + 4 * M, A + 5 * M, A + 4 * M + 256]) == INV  # two output buffers overlap
+    assert call(outs=[A + 4 * M, A + 5 * M, A + 3 * M]) == INV  # an output buffer overlaps the lists
+    assert call(outs=[A + 4 * M, A + 4 * M, A + 6 * M]) != INV  # an empty range may share an address
     assert call(h0=3) == INV                        # heads past out_heads
     assert call(out_heads=1) == INV
     assert call(h0=-1) == INV
@@ -192,6 +198,7 @@ def test_attention_joint_argument_validation_without_gpu(lib):
     assert call(text=-1) == INV
     assert call(T=1, L=1, P=1 << 30, text=1 << 30) == INV  # video tokens fit, video + text pass INT_MAX
     assert call(out=A + 2 * M + 16) == INV               # output overlaps v
+    assert call(lists=A + 4 * M + 32) == INV             # output overlaps the lists
     assert call(q=0) == INV
     assert call(L=9) == INV
     assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED

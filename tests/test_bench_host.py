@@ -16,7 +16,7 @@ import bench  # noqa: E402
 
 
 def test_flop_model_matches_workload_figures():
-    from block_sparse_attention_frame_b200.synthetic import WORKLOADS
+    from synthetic import WORKLOADS
 
     assert bench.flops_per_call(WORKLOADS["wan1.3b_6x"]) / 1e12 == pytest.approx(37.993, rel=1e-4)
     assert bench.flops_per_call(WORKLOADS["wan14b_6x"]) / 1e12 == pytest.approx(126.64, rel=1e-4)
@@ -44,8 +44,40 @@ def test_reference_arm_json_line(capsys):
     assert rc == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
-    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"].startswith("oracle") and cb["value"] == line["value"]
+    assert cb["cores"] >= 1 and cb["nproc"] >= 1 and "cpu_model" in cb
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"] == "tiny"
+    # ms_per_step is what one step of the arm took (a bounded sample); the full call is extrapolated apart
+    assert 0 < line["ms_per_step"] < 5000
+    assert line["full_call_ms_extrapolated"] > 0
+
+
+def test_reference_arm_does_not_load_the_cuda_library():
+    """The oracle arm imports the input generator and the oracle only: the CUDA library stays unloaded."""
+    code = (
+        "import sys, json; sys.path.insert(0, %r); import bench; "
+        "rc = bench.main(['--impl', 'reference', '--workload', 'tiny', '--steps', '1', '--warmup', '3', "
+        "'--ref-seconds', '0.02']); "
+        "maps = open('/proc/self/maps').read(); "
+        "print('LOADED' if 'liblvsa' in maps else 'NOT_LOADED'); "
+        "print('PKG' if 'block_sparse_attention_frame_b200' in sys.modules else 'NO_PKG')" % ROOT)
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
+                         env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert res.returncode == 0, res.stderr[-2000:]
+    assert "NOT_LOADED" in res.stdout and "NO_PKG" in res.stdout, res.stdout
+
+
+def test_oracle_list_build_timing_and_page_context():
+    t = bench.oracle_list_build_us(steps=3)
+    assert set(t) == set(bench.LIST_CONFIGS)
+    for name, r in t.items():
+        assert (r["T"], r["C"], r["W"]) == bench.LIST_CONFIGS[name]
+        assert 0 < r["median_us"] <= r["max_us"]
+    ctx = bench.PAGES_CONTEXT["end_to_end_generation_single_80GB_gpu"][0]
+    assert (ctx["dense_min"], ctx["lvsa_min"], ctx["speedup"]) == (51, 16, 3.17)
+    info = bench.host_info()
+    assert info["nproc"] >= 1 and info["blas_threads"] >= 1
 
 
 def _free_port():

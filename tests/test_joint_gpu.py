@@ -19,7 +19,7 @@ REL_MEAN = 1e-2
 
 
 def test_no_text_tokens_is_the_video_call_bit_for_bit(gpu_lib):
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     q, k, v = synthetic.make_custom(6, 300, 3, 128, seed=2, device="cuda")
     lists = torch.from_numpy(gpu_lib.lvsa_build_frame_lists(6, 4, 2, 1)).cuda()
@@ -44,7 +44,7 @@ JOINT_CASES = [
 @pytest.mark.parametrize("T,P,n_text,H,d,C,W,step,B",
                          [c + (1,) for c in JOINT_CASES] + [c + (2,) for c in JOINT_CASES if c[0] * c[1] <= 2000])
 def test_joint_matches_oracle(gpu_lib, T, P, n_text, H, d, C, W, step, B):
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     q, k, v = synthetic.make_joint(T, P, n_text, H, d, B=B, seed=T + n_text, device="cpu")
     lists_np = gpu_lib.lvsa_build_frame_lists(T, C, W, step)
@@ -66,7 +66,7 @@ def test_joint_matches_oracle(gpu_lib, T, P, n_text, H, d, C, W, step, B):
 def test_full_size_joint_call_sampled_rows(gpu_lib):
     """HunyuanVideo-1.5 1.5x shape (T = 49, P = 1560, 16 heads) with 256 text tokens: sampled video rows of
     five frames and sampled text rows against the oracle."""
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     T, P, n_text, H, d, C, W, step = 49, 1560, 256, 16, 128, 33, 13, 7
     q, k, v = synthetic.make_joint(T, P, n_text, H, d, seed=1005, device="cuda")
@@ -81,11 +81,12 @@ def test_full_size_joint_call_sampled_rows(gpu_lib):
     rows += [T * P, T * P + n_text - 1] + list(T * P + g.choice(n_text, 14, replace=False))
     rows = sorted(set(int(r) for r in rows))
     lists = OL.frame_lists(T, C, W, step)
-    ref = OA.joint_attention_rows(q, k, v, lists, P, T, rows)
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()  # the oracle takes host tensors
+    ref = OA.joint_attention_rows(qc, kc, vc, lists, P, T, rows)
     got = out[:, rows].float().cpu().numpy()
     err = np.abs(got - ref)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
     assert err.mean() <= REL_MEAN * np.abs(ref).mean(), (err.mean(), np.abs(ref).mean())
-    wrong = OA.joint_attention_rows(q, k, v, OL.frame_lists(T, C, W, step + 1), P, T, rows)
+    wrong = OA.joint_attention_rows(qc, kc, vc, OL.frame_lists(T, C, W, step + 1), P, T, rows)
     video = [i for i, r in enumerate(rows) if r < T * P]
     assert np.abs(got[:, video] - wrong[:, video]).mean() > 10 * REL_MEAN * np.abs(ref).mean()

@@ -65,3 +65,20 @@ def test_random_parameters_bit_exact(lib):
         W = int(g.integers(1, C + 1))
         s = int(g.integers(0, 10**9))
         assert lib.lvsa_build_frame_lists(T, C, W, s).tolist() == OL.frame_lists(T, C, W, s), (T, C, W, s)
+
+
+def test_pipeline_lists_rotating_and_fixed_grid(lib):
+    """The per-step pipeline's host lists: step s's lists when the anchors rotate; the step-0 lists at every
+    step in the fixed-grid ablation (anchors that never move)."""
+    from block_sparse_attention_frame_b200 import pipeline
+
+    T, C, W = 121, 21, 9
+    step0 = OL.frame_lists(T, C, W, 0)
+    for s in range(50):
+        rot = pipeline.host_lists(T, C, W, s)
+        fixed = pipeline.host_lists(T, C, W, s, fixed_grid=True)
+        assert rot.tolist() == OL.frame_lists(T, C, W, s)
+        assert fixed.tolist() == step0
+        assert pipeline.list_step(s, True) == 0 and pipeline.list_step(s, False) == s
+        if s % T != 0:
+            assert rot.tolist() != step0

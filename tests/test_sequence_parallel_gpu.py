@@ -55,7 +55,7 @@ def same_bits(a, b):
 
 
 def test_tiny_workload_emulated_ranks_match_single_call_and_oracle(gpu_lib):
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     w = synthetic.WORKLOADS["tiny"]
     q, k, v = synthetic.make_qkv(w, device="cpu")
@@ -81,7 +81,7 @@ def test_tiny_workload_emulated_ranks_match_single_call_and_oracle(gpu_lib):
     (9, 200, 2, 64, 1, 5, 2, [1, 1799]),                 # d = 64, a one-token range
 ])
 def test_emulated_ranks_match_single_call(gpu_lib, T, P, H, d, B, C, W, chunks):
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     q, k, v = synthetic.make_custom(T, P, H, d, B=B, seed=T * 31 + H, device="cuda")
     lists = torch.from_numpy(gpu_lib.lvsa_build_frame_lists(T, C, W, 3)).cuda()
@@ -92,7 +92,7 @@ def test_emulated_ranks_match_single_call(gpu_lib, T, P, H, d, B, C, W, chunks):
 
 def test_routed_call_writes_only_its_heads(gpu_lib):
     """Heads outside [head0, head0 + heads) of the output rows stay as they were."""
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     T, P, H, d = 5, 256, 4, 128
     q, k, v = synthetic.make_custom(T, P, H, d, seed=5, device="cuda")
@@ -120,7 +120,7 @@ sys.path.insert(0, {root!r})
 import torch
 import torch.distributed as dist
 import block_sparse_attention_frame_b200 as lvsa
-from block_sparse_attention_frame_b200 import synthetic
+import synthetic
 from block_sparse_attention_frame_b200.sequence_parallel import SequenceParallelAttention
 
 rank = int(os.environ["RANK"])
@@ -195,7 +195,7 @@ def test_rows_routed_to_host_memory_take_the_system_scope_path(gpu_lib):
     """A range buffer that is not this GPU's memory (here pinned host memory, which the GPU addresses
     directly) makes the kernel release its stores at system scope, the path peer stores take; the rows
     written there equal the single call's."""
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     T, P, H, d = 6, 300, 2, 128
     q, k, v = synthetic.make_custom(T, P, H, d, seed=13, device="cuda")
@@ -214,7 +214,7 @@ def test_rows_routed_to_host_memory_take_the_system_scope_path(gpu_lib):
 def test_unaddressable_range_buffer_is_refused(gpu_lib):
     """Pageable host memory cannot be written by the GPU: the call returns an argument error before any
     launch."""
-    from block_sparse_attention_frame_b200 import synthetic
+    import synthetic
 
     T, P, H, d = 4, 256, 1, 128
     q, k, v = synthetic.make_custom(T, P, H, d, seed=3, device="cuda")
@@ -224,3 +224,22 @@ def test_unaddressable_range_buffer_is_refused(gpu_lib):
     with pytest.raises(gpu_lib.LvsaError) as e:
         gpu_lib.lvsa_attention_to_chunks(q, k, v, lists, P, [dev_part, pageable.data_ptr()], [512, 512], H, 0)
     assert e.value.status == gpu_lib.LVSA_ERR_INVALID_ARG
+
+
+def test_unaddressable_source_range_is_refused(gpu_lib):
+    """The gather reads every source range from the GPU: a pageable host buffer among them is refused with an
+    argument error before any launch; the same range in pinned (mapped) host memory is read like any other."""
+    T, P, H, d = 4, 256, 2, 128
+    src = [torch.randn((1, 512, H, d), device="cuda").to(torch.bfloat16) for _ in range(3)]
+    pageable = [torch.randn((1, 512, H, d)).to(torch.bfloat16) for _ in range(3)]
+    bands = [torch.empty((1, 1024, 1, d), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    tables = [[s, p.data_ptr()] for s, p in zip(src, pageable)]
+    with pytest.raises(gpu_lib.LvsaError) as e:
+        gpu_lib.lvsa_seq_to_heads(*tables, [512, 512], 1, 1, *bands, heads=H)
+    assert e.value.status == gpu_lib.LVSA_ERR_INVALID_ARG
+    pinned = [p.pin_memory() for p in pageable]
+    gpu_lib.lvsa_seq_to_heads(*[[s, p.data_ptr()] for s, p in zip(src, pinned)], [512, 512], 1, 1, *bands, heads=H)
+    torch.cuda.synchronize()
+    for b, s, p in zip(bands, src, pinned):
+        want = torch.cat([s[:, :, 1:2], p.cuda()[:, :, 1:2]], dim=1)
+        assert torch.equal(b.view(torch.int16), want.view(torch.int16))
