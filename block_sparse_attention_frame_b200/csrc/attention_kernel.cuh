@@ -641,40 +641,45 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         mbar_arrive(bar_p + qi);
         ++j;
       }
-      if (ok && j > 0) {
-        ok = __all_sync(0xffffffffu, wait_bounded(bar_o + qi, (j - 1) & 1, w));
-        if (ok) {
-          tc_fence_after();
-          const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a frame with no valid list entry: zero output
-          const bool valid = row < r1;
-          // the buffer that holds this row's token: the last chunk starting at or before it (an empty
-          // chunk is never that one, since the next chunk starts at the same token)
-          int c = 0;
-          for (int hi = p.nchunks - 1; c < hi;) {
-            const int mid = (c + hi + 1) >> 1;
-            if (p.chunk_start[mid] <= row) c = mid; else hi = mid - 1;
-          }
-          const int c0 = p.chunk_start[c];
-          const size_t clen = static_cast<size_t>(p.chunk_start[c + 1] - c0);
-          __nv_bfloat16* dst = p.out_chunk[c] + ((b * clen + (row - c0)) * p.HS + p.head0 + h) * D;
+      // j == 0: the block walked no tile at all (its frames have no valid list entry); O in TMEM was never
+      // written, and the rows get zeros
+      if (ok && j > 0) ok = __all_sync(0xffffffffu, wait_bounded(bar_o + qi, (j - 1) & 1, w));
+      if (ok) {
+        if (j > 0) tc_fence_after();
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a frame with no valid list entry: zero output
+        const bool valid = row < r1;
+        // the buffer that holds this row's token: the last chunk starting at or before it (an empty
+        // chunk is never that one, since the next chunk starts at the same token)
+        int c = 0;
+        for (int hi = p.nchunks - 1; c < hi;) {
+          const int mid = (c + hi + 1) >> 1;
+          if (p.chunk_start[mid] <= row) c = mid; else hi = mid - 1;
+        }
+        const int c0 = p.chunk_start[c];
+        const size_t clen = static_cast<size_t>(p.chunk_start[c + 1] - c0);
+        __nv_bfloat16* dst = p.out_chunk[c] + ((b * clen + (row - c0)) * p.HS + p.head0 + h) * D;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          if (j > 0) {
             tmem_ld32(o_tmem + 32 * c, o);
             tmem_wait_ld_regs(o);
-            if (valid) {
-              uint4 pk[4];
-              uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+          } else {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) pw[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
-              uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) d4[i] = pk[i];
-            }
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
           }
-          // stores into another GPU's memory: ordered before anything the host does after this kernel
-          if (p.routed) __threadfence_system();
+          if (valid) {
+            uint4 pk[4];
+            uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pw[i] = pack_bf16x2(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = pk[i];
+          }
         }
+        // stores into another GPU's memory: ordered before anything the host does after this kernel
+        if (p.routed) __threadfence_system();
       }
     }
   }

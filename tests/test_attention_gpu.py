@@ -249,6 +249,26 @@ def test_frame_without_valid_entries_gives_zeros(gpu_lib):
     assert_close(out[:, rows], ref, "other frames")
 
 
+@pytest.mark.parametrize("T,P,d", [(4, 512, 128), (5, 100, 64)])
+def test_blocks_with_no_listed_frame_write_zeros(gpu_lib, T, P, d):
+    """Query blocks that lie wholly inside a frame with no valid list entry walk no K/V tile at all: their
+    rows are still written, as zeros, whatever the output buffer held (P = 512: 256-row blocks aligned to
+    the frames; P = 100: one block per frame)."""
+    q, k, v = make(T, P, 2, d, seed=17)
+    gpu_lib.lvsa_get_device_status(clear=True)
+    lists = gpu_lib.lvsa_build_frame_lists(T, 3, 1, 2).copy()
+    lists[1, :] = -1
+    out = torch.full_like(q, float("nan"))
+    gpu_lib.lvsa_attention(q, k, v, torch.from_numpy(lists).cuda(), P, out=out)
+    torch.cuda.synchronize()
+    assert gpu_lib.lvsa_get_device_status(clear=True) & gpu_lib.LVSA_DEV_BAD_LIST
+    got = full_out(out)
+    assert np.all(got[:, P:2 * P] == 0)
+    rows = [r for r in range(T * P) if r // P != 1]
+    ref = OA.sparse_attention_rows(*host(q, k, v), [list(r) for r in lists], P, rows)
+    assert_close(got[:, rows], ref, "other frames")
+
+
 def run_host_path(lib, q, k, v, lists_np, P, heads_per_band=0, scale=0.0):
     """The host-buffer entry point: CPU tensors in, CPU tensor out, staging buffers on the GPU."""
     qh, kh, vh = (x.cpu().contiguous().pin_memory() for x in (q, k, v))
