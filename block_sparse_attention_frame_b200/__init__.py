@@ -12,6 +12,8 @@ Functions carry the C ABI's names (declared in ``include/lvsa.h``):
 ``lvsa_attention_joint(q, k, v, lists, tokens_per_frame, scale=0, out=None, stream=None)`` (video + text)
 ``lvsa_attention_host(q_host, k_host, v_host, lists_host, tokens_per_frame, out_host, q_dev, k_dev, v_dev,
 lists_dev, out_dev, scale=0, heads_per_band=0, stream=None)``
+``lvsa_attention_host_static(q_host, k_host, v_host, lists_host, tokens_per_frame, out_host, scale=0, stream=None)``
+(no allocation, no caller device buffer)
 ``lvsa_seq_to_heads(q_chunks, k_chunks, v_chunks, chunk_tokens, head0, band, q_band, k_band, v_band, stream=None)``
 ``lvsa_attention_to_chunks(q, k, v, lists, tokens_per_frame, out_chunks, chunk_tokens, out_heads, head0, scale=0,
 stream=None)``
@@ -40,12 +42,13 @@ LVSA_ERR_BAD_LIST = 6
 LVSA_DEV_TIMEOUT = 0x1
 LVSA_DEV_BAD_LIST = 0x2
 LVSA_IPC_HANDLE_BYTES = 72
+LVSA_STATIC_SCRATCH_BYTES = 64 << 20
 
 EXPORTED = [
     "lvsa_build_frame_lists", "lvsa_build_anchors", "lvsa_attention", "lvsa_attention_host", "lvsa_get_device_status",
     "lvsa_set_wait_budget_ns", "lvsa_watchdog_selftest", "lvsa_status_string",
     "lvsa_version", "lvsa_seq_to_heads", "lvsa_attention_to_chunks", "lvsa_ipc_export", "lvsa_ipc_import",
-    "lvsa_ipc_release", "lvsa_attention_joint",
+    "lvsa_ipc_release", "lvsa_attention_joint", "lvsa_attention_host_static",
 ]
 
 
@@ -78,6 +81,9 @@ _lib.lvsa_attention_joint.restype = _c_int
 _lib.lvsa_attention_host.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_float, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_vp]
 _lib.lvsa_attention_host.restype = _c_int
+_lib.lvsa_attention_host_static.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                            _c_int, _c_float, _c_vp, _c_vp]
+_lib.lvsa_attention_host_static.restype = _c_int
 _lib.lvsa_seq_to_heads.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                    _c_vp, _c_vp, _c_vp, _c_vp]
 _lib.lvsa_seq_to_heads.restype = _c_int
@@ -288,6 +294,44 @@ def lvsa_attention_host_raw(*args) -> int:
     a[10] = float(a[10])
     a[18] = ctypes.c_void_p(a[18])
     return int(_lib.lvsa_attention_host(*a))
+
+
+def lvsa_attention_host_static(q_host, k_host, v_host, lists_host, tokens_per_frame: int, out_host,
+                               scale: float = 0.0, stream=None):
+    """Block-sparse attention on host tensors with no allocation and no caller device buffer: the library
+    stages everything in its own static device array (LVSA_STATIC_SCRATCH_BYTES per GPU), for callers that
+    cannot allocate device memory.  q_host, k_host, v_host, out_host: CPU bf16 [batch, T*tokens_per_frame,
+    heads, d], contiguous (pinned for asynchronous copies); lists_host: CPU int32 [T, L].  Runs on ``stream``
+    of the current CUDA device (default: its current torch stream); synchronise before reading out_host.
+    Calls that overlap on the GPU share the array and race: serialise them."""
+    import torch
+
+    for name, x in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host), ("out_host", out_host)):
+        if not isinstance(x, torch.Tensor) or x.device.type != "cpu" or x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a CPU bfloat16 tensor")
+        if not x.is_contiguous() or x.dim() != 4 or x.shape != q_host.shape:
+            raise ValueError(f"{name} must be contiguous [batch, tokens, heads, d] shaped like q_host")
+    if (lists_host.device.type != "cpu" or lists_host.dtype != torch.int32 or lists_host.dim() != 2
+            or not lists_host.is_contiguous()):
+        raise TypeError("lists_host must be a contiguous CPU int32 tensor [T, L]")
+    B, ntok, H, d = q_host.shape
+    T, L = lists_host.shape
+    if ntok != T * tokens_per_frame:
+        raise ValueError(f"q_host has {ntok} tokens, expected T*tokens_per_frame = {T * tokens_per_frame}")
+    dev = torch.cuda.current_device()
+    st = _lib.lvsa_attention_host_static(q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(),
+                                         lists_host.data_ptr(), L, T, tokens_per_frame, H, d, B, float(scale),
+                                         out_host.data_ptr(), _stream_ptr(stream, dev))
+    _check("lvsa_attention_host_static", st)
+    return out_host
+
+
+def lvsa_attention_host_static_raw(*args) -> int:
+    """The C call with raw pointers (13 arguments in the header's order); returns the status unchanged."""
+    a = list(args)
+    a[10] = float(a[10])
+    a[12] = ctypes.c_void_p(a[12])
+    return int(_lib.lvsa_attention_host_static(*a))
 
 
 def _addr(x) -> int:

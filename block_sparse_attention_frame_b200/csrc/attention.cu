@@ -464,6 +464,78 @@ extern "C" lvsa_status lvsa_attention_host(const void* q_host, const void* k_hos
   return LVSA_OK;
 }
 
+// ------------------------------------------------------------------ staging without allocation
+// lvsa_attention_host_static stages its inputs and output in this array instead of caller buffers or
+// allocations.  In host code `g_static_scratch` names a host-side stand-in, not device memory: the device
+// address is looked up once per device with cudaGetSymbolAddress (that device current) and kept.
+namespace lvsa {
+namespace {
+constexpr size_t kStaticScratchBytes = LVSA_STATIC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_base[64] = {};
+
+size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// The array's device address on device `dev` (the current device); null if CUDA cannot give it.
+void* static_scratch(int dev) {
+  std::lock_guard<std::mutex> g(g_static_mu);
+  if (!g_static_base[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    g_static_base[dev] = ptr;
+  }
+  return g_static_base[dev];
+}
+}  // namespace
+}  // namespace lvsa
+
+extern "C" lvsa_status lvsa_attention_host_static(const void* q_host, const void* k_host, const void* v_host,
+                                                  const int32_t* lists_host, int L, int T, int tokens_per_frame,
+                                                  int heads, int d, int batch, float scale, void* out_host,
+                                                  void* stream) {
+  using namespace lvsa;
+  const int P = tokens_per_frame;
+  if (!q_host || !k_host || !v_host || !lists_host || !out_host) return LVSA_ERR_INVALID_ARG;
+  if (T < 1 || P < 1 || heads < 1 || batch < 1 || L < 1 || L > T) return LVSA_ERR_INVALID_ARG;
+  const lvsa_status cs = check_sizes(L, T, P, heads, d, batch, scale);
+  if (cs != LVSA_OK) return cs;
+  const size_t bytes = static_cast<size_t>(batch) * T * P * heads * static_cast<size_t>(d) * 2;
+  const size_t list_bytes = static_cast<size_t>(T) * L * 4;
+  if (!disjoint(out_host, q_host, bytes) || !disjoint(out_host, k_host, bytes) || !disjoint(out_host, v_host, bytes) ||
+      !ranges_disjoint(out_host, bytes, lists_host, list_bytes))
+    return LVSA_ERR_INVALID_ARG;
+  // layout in the array: Q, K, V, output, lists, each at a 256-byte boundary
+  const size_t slot = round256(bytes);
+  if (slot > kStaticScratchBytes / 4 || 4 * slot + round256(list_bytes) > kStaticScratchBytes)
+    return LVSA_ERR_INVALID_ARG;
+  int dev = 0;
+  const lvsa_status ds = check_device(&dev);
+  if (ds != LVSA_OK) return ds;
+  if (dev >= 64) return LVSA_ERR_UNSUPPORTED;
+  char* base = static_cast<char*>(static_scratch(dev));
+  if (!base) return LVSA_ERR_CUDA;
+  char* q_d = base;
+  char* k_d = base + slot;
+  char* v_d = base + 2 * slot;
+  char* out_d = base + 3 * slot;
+  int32_t* lists_d = reinterpret_cast<int32_t*>(base + 4 * slot);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const struct { void* dst; const void* src; size_t n; } up[4] = {
+      {lists_d, lists_host, list_bytes}, {q_d, q_host, bytes}, {k_d, k_host, bytes}, {v_d, v_host, bytes}};
+  for (const auto& c : up)
+    if (cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, st) != cudaSuccess) return LVSA_ERR_CUDA;
+  const lvsa_status r = launch_band(q_d, k_d, v_d, lists_d, L, T, P, heads, heads, d, batch, scale,
+                                    one_buffer(out_d, static_cast<long long>(T) * P, heads), st, dev);
+  if (r != LVSA_OK) return r;
+  if (cudaMemcpyAsync(out_host, out_d, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return LVSA_ERR_CUDA;
+  return LVSA_OK;
+}
+
 extern "C" lvsa_status lvsa_get_device_status(unsigned int* flags, int clear) {
   if (!flags) return LVSA_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return LVSA_ERR_CUDA;

@@ -190,6 +190,50 @@ lvsa_status lvsa_attention_host(const void* q_host, const void* k_host, const vo
                                 void* q_dev, void* k_dev, void* v_dev, int32_t* lists_dev,
                                 void* out_dev, int heads_per_band, void* stream);
 
+/* Bytes of the device staging array lvsa_attention_host_static works in (64 MiB). */
+#define LVSA_STATIC_SCRATCH_BYTES (64ull << 20)
+
+/*
+ * lvsa_attention_host_static -- lvsa_attention on HOST inputs and output that
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library call,
+ * and no caller-provided device buffer.
+ *
+ * The paper has no counterpart to this call.  It is for callers that cannot
+ * get device memory of their own for staging: a plug-in running inside a
+ * process whose allocator already owns the GPU's memory (a framework's caching
+ * allocator, or a memory-capped service), or code on a path where cudaMalloc /
+ * cudaFree must not be called because they can block or synchronise the whole
+ * device.
+ *
+ * The inputs, the lists and the output are staged in one array of
+ * LVSA_STATIC_SCRATCH_BYTES in the library's own device memory (a static
+ * __device__ array: every GPU that loads the library holds it until the
+ * process exits).  Q, K, V, the lists and the output are copied host -> array
+ * -> host on `stream` around one attention launch; the result is the one
+ * lvsa_attention computes.
+ *
+ * Arguments: q_host, k_host, v_host, lists_host, L, T, tokens_per_frame, heads,
+ *   d, batch, scale, out_host as lvsa_attention_host (host buffers; pinned
+ *   memory lets the copies run asynchronously); stream a cudaStream_t (as
+ *   void*), NULL = default stream.
+ * Limit: 4 * batch*T*tokens_per_frame*heads*d*2 bytes (Q, K, V, output, each
+ *   rounded up to 256 bytes) + T*L*4 bytes (lists, rounded up to 256) must fit
+ *   in LVSA_STATIC_SCRATCH_BYTES; a larger call is refused with
+ *   LVSA_ERR_INVALID_ARG before anything is copied or launched.
+ * Behaviour: asynchronous on `stream`; synchronise it before reading out_host.
+ *   The first call on a device looks up the array's device address (one
+ *   cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  Every call on a device shares the one array,
+ *   which keeps the previous call's contents (each call overwrites what it
+ *   reads before reading it): calls whose work overlaps on the GPU (other
+ *   streams, other host threads) race on it -- serialise them, e.g. on one
+ *   stream.  Errors as lvsa_attention.
+ */
+lvsa_status lvsa_attention_host_static(const void* q_host, const void* k_host, const void* v_host,
+                                       const int32_t* lists_host, int L, int T, int tokens_per_frame,
+                                       int heads, int d, int batch, float scale, void* out_host,
+                                       void* stream);
+
 /*
  * Sequence-parallel use (DeepSpeed-Ulysses layout, under which the method runs
  * Wan 2.2-A14B on 8 NPUs: techwalker article, section 五).  N ranks, one per
