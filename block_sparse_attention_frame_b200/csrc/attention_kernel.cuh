@@ -20,7 +20,11 @@
 //   warps 0-3   softmax of query tile 0, warps 4-7 of query tile 1, one thread per row (TMEM lane):
 //               online softmax in the exp2 domain with a lazily updated running max (O in TMEM is
 //               rescaled only when the max grows by more than 2^8), P written back over the S columns
-//               as bf16; rows of the other frame skip the tiles their frame does not attend.
+//               as bf16; rows of the other frame skip the tiles their frame does not attend.  On full
+//               tiles the exponentials start with the running max as soon as the first 32 columns of S
+//               are loaded, and the tile max is computed alongside them (a row whose max grew by more
+//               than 2^8 has its first 64 keys redone), so neither the rest of the load nor the max
+//               waits in front of the exponentials.
 //               Epilogue O / l -> bf16 -> HBM.  The output rows may be split by token range over several
 //               buffers, other GPUs' included (sequence-parallel use): each row is stored straight into
 //               the buffer of the rank that owns its tokens, so the attention and the head-to-sequence
@@ -48,10 +52,10 @@ constexpr int kBM = 128;          // query rows per tile = MMA M
 constexpr int kBN = 128;          // keys per K/V tile = largest MMA N of QK^T
 constexpr int kQTiles = 2;        // query tiles per CTA, sharing every K/V tile
 constexpr int kThreads = 384;     // warps 0-3: softmax tile 0, 4-7: softmax tile 1, 8: TMA, 9: MMA, 10-11 idle
-// Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup drops to 88 and the
-// two softmax warpgroups rise to 208: 2 x 128 x 208 + 128 x 88 = 64512.
-constexpr uint32_t kRegsSoftmax = 208;
-constexpr uint32_t kRegsControl = 88;
+// Registers: launched at 168 per thread (384 x 168 = 64512); the TMA/MMA warpgroup drops to 56 and the
+// two softmax warpgroups rise to 224: 2 x 128 x 224 + 128 x 56 = 64512 (the softmax then needs no spill).
+constexpr uint32_t kRegsSoftmax = 224;
+constexpr uint32_t kRegsControl = 56;
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr int kTmemCols = 512;    // S/P of tile i: columns [128 i, 128 i + 128); O of tile i: [256 + 128 i, ...)
@@ -216,6 +220,36 @@ struct FrameWalk {
 };
 
 // ------------------------------------------------------------------ softmax of one S tile
+// Exponentials of chunk c (32 keys) of the row: P as bf16 pairs over the S columns, row sum into acc.
+__device__ __forceinline__ void exp_store_chunk(uint32_t s_tmem, const float* sc, float2 scale2, float2 negm2,
+                                                float2* acc, int c) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 x = ffma2(make_float2(sc[2 * i], sc[2 * i + 1]), scale2, negm2);
+    float2 e;
+    e.x = ex2(x.x);
+    e.y = ex2(x.y);
+    acc[i & 3] = fadd2(acc[i & 3], e);
+    pk[i] = pack_bf16x2(e.x, e.y);
+  }
+  tmem_st16(s_tmem + 16 * c, pk);
+}
+
+__device__ __forceinline__ float row_max128(const float* s) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = s[k];
+#pragma unroll
+  for (int i = 8; i < 120; i += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 8 + k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[120 + k]);
+  return fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7]));
+}
+
 // Thread = one query row.  Loads the row of S from TMEM, masks columns past the
 // run end, updates the running max lazily (rescaling the row of O in TMEM when
 // needed), writes P = 2^(scale*log2e*s - m) as bf16 over the S columns and
@@ -227,6 +261,65 @@ template <int D>
 __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int nv, int j, bool skip, float sl2,
                                              float& m, float& l, uint64_t* bar_o, const Watch& w, uint64_t* bar_half) {
   float s[kBN];
+  // Speculative path (full tiles, every row of the warp with a finite running max or skipping the tile):
+  // the exponentials start with the running max as soon as keys 0..31 are loaded, and the tile max is
+  // computed alongside; a warp with a row whose max grew by more than 2^8 redoes keys 0..63 with the new
+  // max before handing them over.
+  if (nv == kBN && __all_sync(0xffffffffu, m != -INFINITY || skip)) {
+    const float2 scale2 = make_float2(sl2, sl2);
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    tmem_ld32(s_tmem + 0, s + 0);
+    tmem_wait_ld_regs(s + 0);
+    tmem_ld32(s_tmem + 32, s + 32);
+    tmem_ld32(s_tmem + 64, s + 64);
+    tmem_ld32(s_tmem + 96, s + 96);
+    float2 negm2 = skip ? make_float2(-INFINITY, -INFINITY) : make_float2(-m, -m);
+    exp_store_chunk(s_tmem, s + 0, scale2, negm2, acc, 0);
+    tmem_wait_ld_regs(s + 32);
+    tmem_wait_ld_regs(s + 64);
+    tmem_wait_ld_regs(s + 96);
+    const float tile_max = skip ? -INFINITY : row_max128(s) * sl2;
+    exp_store_chunk(s_tmem, s + 32, scale2, negm2, acc, 1);
+    if (__any_sync(0xffffffffu, tile_max > m + kRescaleLog2)) {
+      float alpha = 1.f;
+      if (tile_max > m + kRescaleLog2) {
+        alpha = ex2(m - tile_max);
+        l *= alpha;
+        m = tile_max;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!__all_sync(0xffffffffu, wait_bounded(bar_o, (j - 1) & 1, w))) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(o_tmem + 32 * c, o);
+          tmem_wait_ld_regs(o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(o_tmem + 32 * c, o);
+        }
+      }
+      // keys 0..63 again with the new max (after the first stores of those columns have completed)
+      tmem_wait_st();
+      negm2 = skip ? make_float2(-INFINITY, -INFINITY) : make_float2(-m, -m);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+      exp_store_chunk(s_tmem, s + 0, scale2, negm2, acc, 0);
+      exp_store_chunk(s_tmem, s + 32, scale2, negm2, acc, 1);
+    }
+    // keys 0..63 of P are in TMEM: the MMA warp may start the first half of PV
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar_half);
+    exp_store_chunk(s_tmem, s + 64, scale2, negm2, acc, 2);
+    exp_store_chunk(s_tmem, s + 96, scale2, negm2, acc, 3);
+    const float2 t01 = fadd2(acc[0], acc[1]);
+    const float2 t23 = fadd2(acc[2], acc[3]);
+    const float2 tt = fadd2(t01, t23);
+    l += tt.x + tt.y;
+    return true;
+  }
   tmem_ld32(s_tmem + 0, s + 0);
   if (nv > 32) tmem_ld32(s_tmem + 32, s + 32);
   if (nv > 64) tmem_ld32(s_tmem + 64, s + 64);
@@ -434,10 +527,10 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     }
     __syncwarp();
     int issued = 0;
+    int slot = 0;         // ring slot and phase of the next load
+    uint32_t phase = 0;
     bool ok = true;
     auto load = [&](const CUtensorMap* tm, int tok) {
-      const int slot = issued % Cf::kSlots;
-      const uint32_t phase = (issued / Cf::kSlots) & 1;
       if (!__all_sync(0xffffffffu, wait_bounded(bar_empty + slot, phase ^ 1, w))) {
         ok = false;
         return;
@@ -451,6 +544,10 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       }
       __syncwarp();
       ++issued;
+      if (++slot == Cf::kSlots) {
+        slot = 0;
+        phase ^= 1;
+      }
     };
     // consumption order of the MMA warp: K0, V0, K1, V1, ...
     FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
@@ -505,23 +602,32 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       }
     };
     auto commit = [&](uint64_t* bar) { mma_commit(bar); };
-    auto slot_of = [&](int idx) { return idx % Cf::kSlots; };
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wait_bounded(bar, parity, w));
     };
-    auto wait_full = [&](int idx) { return wait_all(bar_full + slot_of(idx), (idx / Cf::kSlots) & 1); };
-
-    int cidx = 0;
+    // ring slot and phase of the next load consumed, advanced by one per load (consumption order K0, V0, K1, ...)
+    int rslot = 0;
+    uint32_t rphase = 0;
+    auto take = [&](int& slot, uint32_t& phase) {
+      slot = rslot;
+      phase = rphase;
+      if (++rslot == Cf::kSlots) {
+        rslot = 0;
+        rphase ^= 1;
+      }
+    };
     bool ok = wait_all(bar_q, 0);
     FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
     int tok, nv, tmask;
     if (ok && walk.next(tok, nv, tmask)) {
       int n_cur = (nv + 15) & ~15;
-      const int k0 = cidx++;
-      ok = wait_full(k0);
+      int k0;
+      uint32_t k0p;
+      take(k0, k0p);
+      ok = wait_all(bar_full + k0, k0p);
       if (ok) {
         tc_fence_after();
-        const uint32_t k_addr = sr + slot_of(k0) * Cf::kTileBytes;
+        const uint32_t k_addr = sr + k0 * Cf::kTileBytes;
         if (elect_one()) {
           qk(0, k_addr, n_cur);
           commit(bar_s + 0);
@@ -529,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
             qk(1, k_addr, n_cur);
             commit(bar_s + 1);
           }
-          commit(bar_empty + slot_of(k0));
+          commit(bar_empty + k0);
         }
         __syncwarp();
       }
@@ -537,9 +643,11 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         int tok_n, nv_n, tmask_n;
         const bool has_next = walk.next(tok_n, nv_n, tmask_n);
         const int n_next = (nv_n + 15) & ~15;
-        const int vi = cidx++;
-        const uint32_t v_addr = sr + slot_of(vi) * Cf::kTileBytes;
-        if (!wait_all(bar_ph + 0, j & 1) || !wait_full(vi)) {
+        int vi;
+        uint32_t vph;
+        take(vi, vph);
+        const uint32_t v_addr = sr + vi * Cf::kTileBytes;
+        if (!wait_all(bar_ph + 0, j & 1) || !wait_all(bar_full + vi, vph)) {
           ok = false;
           break;
         }
@@ -552,9 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         int ki = -1;
         uint32_t k_addr = 0;
         if (has_next) {
-          ki = cidx++;
-          k_addr = sr + slot_of(ki) * Cf::kTileBytes;
-          if (!wait_full(ki)) {
+          uint32_t kph;
+          take(ki, kph);
+          k_addr = sr + ki * Cf::kTileBytes;
+          if (!wait_all(bar_full + ki, kph)) {
             ok = false;
             break;
           }
@@ -572,8 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
           }
           commit(bar_o + 0);
           if (!has1) {
-            commit(bar_empty + slot_of(vi));
-            if (has_next) commit(bar_empty + slot_of(ki));
+            commit(bar_empty + vi);
+            if (has_next) commit(bar_empty + ki);
           }
         }
         __syncwarp();
@@ -597,8 +706,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
               commit(bar_s + 1);
             }
             commit(bar_o + 1);
-            commit(bar_empty + slot_of(vi));
-            if (has_next) commit(bar_empty + slot_of(ki));
+            commit(bar_empty + vi);
+            if (has_next) commit(bar_empty + ki);
           }
           __syncwarp();
         }
