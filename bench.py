@@ -596,16 +596,15 @@ def run_sequence_parallel(args, rank, world, local):
     if lvsa.lvsa_get_device_status(clear=True):
         raise RuntimeError("device status set after the timed region")
 
-    # end to end: this rank's token range of Q, K, V from pinned host memory, its output rows back
+    # end to end: this rank's token range of Q, K, V from pinned host memory, its output rows back, through
+    # the host-buffer call of the sequence-parallel object (one rank: transfers pipelined by bands of heads)
     qh, kh, vh = (x.cpu().pin_memory() for x in (sp.q, sp.k, sp.v))
     oh = torch.empty(sp.out.shape, dtype=sp.out.dtype).pin_memory()
     e2e_steps = max(3, min(args.steps, 10))
 
     def e2e_step(s):
-        for dst, src in ((sp.q, qh), (sp.k, kh), (sp.v, vh)):
-            dst.copy_(src, non_blocking=True)
-        step(s)
-        oh.copy_(sp.out, non_blocking=True)
+        lvsa.lvsa_build_frame_lists(w.T, w.C, w.W, s, out=pinned[s % nsteps].numpy())
+        sp.host_call(qh, kh, vh, pinned[s % nsteps], oh)
 
     e2e_step(0)
     torch.cuda.synchronize()
@@ -650,7 +649,8 @@ def run_sequence_parallel(args, rank, world, local):
         "e2e": {"value": F_call / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": 3 * w.B * (b - a) * row_bytes + w.T * w.L * 4,
                 "d2h_bytes_per_step": w.B * (b - a) * row_bytes,
-                "call": "SequenceParallelAttention on this rank's token range (pinned host buffers)"},
+                "call": "SequenceParallelAttention.host_call on this rank's token range (pinned host buffers; "
+                        "one rank: lvsa_attention_host, transfers pipelined by bands of heads)"},
         "gpu_launches": args.steps * (2 if world > 1 else 1),
         "clocks": clocks.summary(),
     }

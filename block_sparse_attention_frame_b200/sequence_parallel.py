@@ -22,7 +22,7 @@ ranks before r).  The caller writes its inputs into ``q``, ``k``, ``v`` and read
 
 from __future__ import annotations
 
-from . import (lvsa_attention_to_chunks, lvsa_ipc_export, lvsa_ipc_import, lvsa_ipc_release,
+from . import (lvsa_attention_host, lvsa_attention_to_chunks, lvsa_ipc_export, lvsa_ipc_import, lvsa_ipc_release,
                lvsa_seq_to_heads)
 
 
@@ -87,6 +87,7 @@ class SequenceParallelAttention:
             self.q_band, self.k_band, self.v_band = (alloc((batch, tokens, self.band, d)) for _ in range(3))
         else:
             self.q_band = self.k_band = self.v_band = None  # more ranks than heads: this rank only holds tokens
+        self._lists_dev = None  # device copy of the lists for host_call
         self._ipc = ipc if ipc is not None else CudaIpc()
         self._opened = []
         own = [self.q, self.k, self.v, self.out]
@@ -146,6 +147,27 @@ class SequenceParallelAttention:
         if self.world > 1:
             self._barrier()  # every rank's output rows stored
         return self.out
+
+    def host_call(self, q_host, k_host, v_host, lists_host, out_host, scale: float = 0.0):
+        """One call on host buffers: this rank's token range of Q, K, V (CPU bf16 [batch, n, heads, d], pinned
+        for asynchronous copies) in, its range of the output out.  lists_host: CPU int32 [T, L].  Asynchronous
+        on the current stream: synchronise before reading out_host.
+
+        With one rank the whole call is ``lvsa_attention_host``: uploads and readback pipelined against the
+        kernel by bands of heads, staged in this object's buffers.  With several ranks the range buffers must be
+        complete on every rank before any rank gathers, so the copies go before and after the call."""
+        import torch
+
+        if self._lists_dev is None or tuple(self._lists_dev.shape) != tuple(lists_host.shape):
+            self._lists_dev = torch.empty(tuple(lists_host.shape), dtype=torch.int32, device=self.device)
+        if self.world == 1:
+            return lvsa_attention_host(q_host, k_host, v_host, lists_host, self.P, out_host, self.q, self.k, self.v,
+                                       self._lists_dev, self.out, scale=scale)
+        for dev, host in ((self.q, q_host), (self.k, k_host), (self.v, v_host), (self._lists_dev, lists_host)):
+            dev.copy_(host, non_blocking=True)
+        self(self._lists_dev, scale=scale)
+        out_host.copy_(self.out, non_blocking=True)
+        return out_host
 
     def _unmap(self) -> None:
         while self._opened:

@@ -243,3 +243,24 @@ def test_unaddressable_source_range_is_refused(gpu_lib):
     for b, s, p in zip(bands, src, pinned):
         want = torch.cat([s[:, :, 1:2], p.cuda()[:, :, 1:2]], dim=1)
         assert torch.equal(b.view(torch.int16), want.view(torch.int16))
+
+
+def test_host_call_one_rank_equals_single_call(gpu_lib):
+    """One rank: the host-buffer call of the sequence-parallel object (uploads and readback pipelined by bands of
+    heads) gives the single call's output bit for bit."""
+    import synthetic
+    from block_sparse_attention_frame_b200.sequence_parallel import SequenceParallelAttention
+
+    T, P, H, d, B = 6, 300, 3, 128, 2
+    q, k, v = synthetic.make_custom(T, P, H, d, B=B, seed=61, device="cuda")
+    lists_np = gpu_lib.lvsa_build_frame_lists(T, 3, 1, 4)
+    ref = gpu_lib.lvsa_attention(q, k, v, torch.from_numpy(lists_np).cuda(), P)
+    sp = SequenceParallelAttention(T, P, H, d, batch=B)
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):  # the second call reuses the object's staging buffers
+        oh.zero_()
+        sp.host_call(qh, kh, vh, torch.from_numpy(lists_np).pin_memory(), oh)
+        torch.cuda.synchronize()
+        assert same_bits(oh, ref.cpu())
+    sp.close()
