@@ -22,9 +22,10 @@
 //               rescaled only when the max grows by more than 2^8), P written back over the S columns
 //               as bf16; rows of the other frame skip the tiles their frame does not attend.  On full
 //               tiles the exponentials start with the running max as soon as the first 32 columns of S
-//               are loaded, and the tile max is computed alongside them (a row whose max grew by more
-//               than 2^8 has its first 64 keys redone), so neither the rest of the load nor the max
-//               waits in front of the exponentials.
+//               are loaded; the max of keys 64..127 is computed alongside them, and keys 0..63 are
+//               checked through their row sum (a row whose max grew by more than 2^8 has its first 64
+//               keys redone), so neither the rest of the load nor the max waits in front of the
+//               exponentials.
 //               Epilogue O / l -> bf16 -> HBM.  The output rows may be split by token range over several
 //               buffers, other GPUs' included (sequence-parallel use): each row is stored straight into
 //               the buffer of the rank that owns its tokens, so the attention and the head-to-sequence
@@ -62,6 +63,7 @@ constexpr int kTmemCols = 512;    // S/P of tile i: columns [128 i, 128 i + 128)
 constexpr int kOCol0 = 256;
 constexpr int kChunkBytes = kBM * 128;    // one 128-byte-wide swizzle column of a 128-row tile
 constexpr float kRescaleLog2 = 8.0f;      // rescale O only when the max grows by > 2^8
+constexpr float kRescaleSum = 256.0f;     // 2^kRescaleLog2
 
 constexpr int kMaxT = 4096;               // latent frames supported (frame bitmaps in shared memory)
 constexpr int kMaxChunks = 64;            // output buffers a launch can route rows to (token ranges)
@@ -236,6 +238,20 @@ __device__ __forceinline__ void exp_store_chunk(uint32_t s_tmem, const float* sc
   tmem_st16(s_tmem + 16 * c, pk);
 }
 
+__device__ __forceinline__ float row_max64(const float* s) {
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = s[k];
+#pragma unroll
+  for (int i = 8; i < 56; i += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = fmax3(a[k], s[i + k], s[i + 8 + k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = fmaxf(a[k], s[56 + k]);
+  return fmaxf(fmax3(a[0], a[1], a[2]), fmax3(fmax3(a[3], a[4], a[5]), a[6], a[7]));
+}
+
 __device__ __forceinline__ float row_max128(const float* s) {
   float a[8];
 #pragma unroll
@@ -278,9 +294,16 @@ __device__ __forceinline__ bool softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
     tmem_wait_ld_regs(s + 32);
     tmem_wait_ld_regs(s + 64);
     tmem_wait_ld_regs(s + 96);
-    const float tile_max = skip ? -INFINITY : row_max128(s) * sl2;
+    // keys 64..127: their max; keys 0..63: a key more than 2^8 above the running max makes its P, and so
+    // the row sum of keys 0..63, exceed 2^8 -- only then is their max needed
+    const float hi_max = skip ? -INFINITY : row_max64(s + 64) * sl2;
     exp_store_chunk(s_tmem, s + 32, scale2, negm2, acc, 1);
-    if (__any_sync(0xffffffffu, tile_max > m + kRescaleLog2)) {
+    const float2 lo01 = fadd2(acc[0], acc[1]);
+    const float2 lo23 = fadd2(acc[2], acc[3]);
+    const float2 lo = fadd2(lo01, lo23);
+    const bool check = hi_max > m + kRescaleLog2 || lo.x + lo.y > kRescaleSum;
+    if (__any_sync(0xffffffffu, check)) {
+      const float tile_max = skip ? -INFINITY : fmaxf(row_max64(s) * sl2, hi_max);
       float alpha = 1.f;
       if (tile_max > m + kRescaleLog2) {
         alpha = ex2(m - tile_max);
