@@ -134,6 +134,30 @@ def test_large_logits_rescale_path(gpu_lib):
     assert_close(out, OA.sparse_attention(*host(q, k, v), OL.frame_lists(T, 4, 2, 3), P), "rescale")
 
 
+@pytest.mark.parametrize("key_pos", [5, 40, 70, 127])
+def test_max_jump_inside_a_later_tile(gpu_lib, key_pos):
+    """One key far above everything before it, at position key_pos of a later full tile: for key_pos < 64 the
+    speculative softmax sees it only through the row sum of keys 0..63, for key_pos >= 64 through the max of
+    keys 64..127.  Either way the rows must rescale and match the oracle."""
+    T, P, H, d = 4, 512, 1, 128
+    q, k, v = make(T, P, H, d, seed=90 + key_pos)
+    lists = gpu_lib.lvsa_build_frame_lists(T, T, 1, 0)  # dense: one run of 16 full tiles
+    qf, kf = q.float(), k.float()
+    tok = 5 * 128 + key_pos  # a key in the sixth tile of the walk
+    u = torch.randn(d, generator=torch.Generator().manual_seed(key_pos)).to(qf.device)
+    u = u / u.norm()
+    kf[0, tok, 0, :] = 40.0 * u  # far along a direction that the queries of frame 0 share
+    qf[0, :P, 0, :] += 4.0 * u
+    q, k = qf.to(torch.bfloat16).contiguous(), kf.to(torch.bfloat16).contiguous()
+    out = full_out(run_kernel(gpu_lib, q, k, v, lists, P))
+    ref = OA.sparse_attention(*host(q, k, v), OL.frame_lists(T, T, 1, 0), P)
+    # the key dominates the rows of frame 0: its logit is far above the rest
+    S = (q.float()[0, :P, 0, :] @ k.float()[0, :, 0, :].T) / np.sqrt(d)
+    gap = (S[:, tok] - S[:, :tok].max(dim=1).values).median().item() * 1.4427
+    assert gap > 8, gap
+    assert_close(out, ref, f"max jump at key {key_pos}")
+
+
 def test_unsorted_lists_same_result(gpu_lib):
     T, P, H, d = 8, 150, 2, 128
     q, k, v = make(T, P, H, d, seed=3)
