@@ -33,14 +33,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // A band of H heads out of rows of HS heads: [batch][tokens][HS*d] bf16 starting at `base`
 // (the band's first head) viewed as a 3-D tensor {H*d, tokens, batch} with row pitch HS*d;
-// one box = 64 columns (128 bytes, one swizzle row) x 128 tokens.
-bool make_map(CUtensorMap* tm, const void* base, int B, long long tokens, int H, int HS, int d) {
+// one box = 64 columns (128 bytes, one swizzle row) x `rows` tokens (128: a whole tile; 8: a piece of a tile
+// that spans two runs of frames).
+bool make_map(CUtensorMap* tm, const void* base, int B, long long tokens, int H, int HS, int d, int rows = kBM) {
   auto enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(H) * d, static_cast<cuuint64_t>(tokens),
                         static_cast<cuuint64_t>(B)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(HS) * d * 2, static_cast<cuuint64_t>(tokens) * HS * d * 2};
-  cuuint32_t box[3] = {64, kBM, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -153,8 +154,11 @@ lvsa_status launch_band(const void* q, const void* k, const void* v, const int32
   const long long tokens = static_cast<long long>(T) * P + ntext;
   if (!make_map(&kp.tm_q, q, batch, tokens, heads, in_stride, d) ||
       !make_map(&kp.tm_k, k, batch, tokens, heads, in_stride, d) ||
-      !make_map(&kp.tm_v, v, batch, tokens, heads, in_stride, d))
+      !make_map(&kp.tm_v, v, batch, tokens, heads, in_stride, d) ||
+      !make_map(&kp.tm_k8, k, batch, tokens, heads, in_stride, d, 8) ||
+      !make_map(&kp.tm_v8, v, batch, tokens, heads, in_stride, d, 8))
     return LVSA_ERR_CUDA;
+  kp.pack = (P % 8 == 0 && ntext == 0) ? 1 : 0;
   kp.lists = lists;
   kp.T = T;
   kp.P = P;

@@ -10,8 +10,12 @@
 //   warp 8      TMA producer: both 128-row Q tiles once, then K and V tiles of the frames the block
 //               attends into a 5-slot shared-memory ring.  A block may hold the end of frame fa and the
 //               start of fa + 1; it attends the union of their lists, walked as runs of consecutive
-//               frames (one contiguous token range each, cut into 128-token tiles, the last partial).
-//               The gather is done by TMA coordinates: no mask is ever materialised.
+//               frames (one contiguous token range each, cut into 128-token tiles).  In a block of one
+//               frame every row attends every run, so a tile may span the end of one run and the start of
+//               the next (loaded in 8-row boxes); otherwise each run's last tile is partial.  The gather is
+//               done by TMA coordinates: no mask is ever materialised.  The producer alone walks the lists
+//               and publishes a record per tile (valid keys, membership, last tile) that the MMA and
+//               softmax warps read.
 //   warp 9      TMEM allocator and tcgen05.mma issuer (one elected lane):
 //                 S_i = Q_i K_j^T  into query tile i's S columns (SS form)
 //                 O_i += P_i V_j   with P_i read from TMEM (TS form), in two halves of 64 keys
@@ -88,6 +92,9 @@ struct KernelParams {
   CUtensorMap tm_q;
   CUtensorMap tm_k;
   CUtensorMap tm_v;
+  CUtensorMap tm_k8;  // K and V with 8-row boxes: tiles that span two runs are loaded in 8-row pieces
+  CUtensorMap tm_v8;
+  int pack;           // frames hold a multiple of 8 tokens and there is no text: single-frame blocks pack tiles
   const int32_t* lists;
   int T, P, H, L;    // H: heads in this launch (grid.y)
   int ntext;         // text tokens after the T*P video tokens (joint sequence); 0: video only
@@ -183,7 +190,30 @@ struct FrameWalk {
     return static_cast<int>(((ma[g >> 5] >> (g & 31)) & 1u) | (((mb[g >> 5] >> (g & 31)) & 1u) << 1));
   }
 
+  // tiles of a packed walk may span two runs; the last tile's second run starts at token tok_b after n_a
+  // tokens of the first (n_a == the tile's tokens when it lies in one run)
+  bool pack = false;
+  int tok_b = 0, n_a = 0;
+
   __device__ __forceinline__ bool next(int& tok, int& nvalid, int& tmask) {
+    if (!next_run()) return false;
+    tok = pos;
+    nvalid = min(kBN, end - pos);
+    tmask = mask;
+    pos += nvalid;
+    n_a = nvalid;
+    if (pack && nvalid < kBN && next_run()) {
+      tok_b = pos;
+      const int nb = min(kBN - nvalid, end - pos);
+      pos += nb;
+      nvalid += nb;
+      tmask &= mask;
+    }
+    return true;
+  }
+
+  // makes [pos, end) the rest of the current run or the next non-empty run; false after the last
+  __device__ __forceinline__ bool next_run() {
     while (pos >= end) {
       if (f >= T) {
         if (text_run()) continue;
@@ -213,13 +243,42 @@ struct FrameWalk {
       mask = m0;
       f = f1 + 1;
     }
-    tok = pos;
-    nvalid = min(kBN, end - pos);
-    tmask = mask;
-    pos += nvalid;
     return true;
   }
 };
+
+// ------------------------------------------------------------------ tile records
+// The producer walks the frame lists once and publishes, for K/V tile j, a record at entry j % kMetaSlots:
+// bits 16..31 j mod 2^16, bit 10 "last tile", bits 2..9 valid keys nv (0: the walk holds no tile at all),
+// bits 0..1 the membership mask of the tile's frames.  The producer is at most a few tiles ahead of any
+// reader (the K/V ring bounds it), so 16 entries are never overwritten before they are read.
+constexpr int kMetaSlots = 16;
+__device__ __forceinline__ uint32_t tile_record(int j, int nv, int tmask, bool last) {
+  return (static_cast<uint32_t>(j & 0xffff) << 16) | (last ? 1024u : 0u) | (static_cast<uint32_t>(nv) << 2) |
+         static_cast<uint32_t>(tmask);
+}
+__device__ __forceinline__ int rec_nv(uint32_t r) { return static_cast<int>((r >> 2) & 0xff); }
+__device__ __forceinline__ int rec_mask(uint32_t r) { return static_cast<int>(r & 3); }
+__device__ __forceinline__ bool rec_last(uint32_t r) { return (r & 1024u) != 0; }
+
+// Waits (bounded) until tile j's record is published; false when the budget ran out or the CTA gave up.
+__device__ __forceinline__ bool read_record(volatile uint32_t* meta, int j, const Watch& w, uint32_t& rec) {
+  rec = meta[j % kMetaSlots];
+  if ((rec >> 16) == static_cast<uint32_t>(j & 0xffff)) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 1;; ++it) {
+    rec = meta[j % kMetaSlots];
+    if ((rec >> 16) == static_cast<uint32_t>(j & 0xffff)) return true;
+    if ((it & 63u) == 0) {
+      if (*w.abort_flag) return false;
+      if (clock64() - t0 > w.budget_cycles) {
+        *w.abort_flag = 1;
+        atomicOr(&g_lvsa_dev_status, LVSA_DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
 
 // ------------------------------------------------------------------ softmax of one S tile
 // Exponentials of chunk c (32 keys) of the row: P as bf16 pairs over the S columns, row sum into acc.
@@ -444,6 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   uint64_t* bar_ph = bar_o + 2;              // [2] P_i(j) keys 0..63 written (128 arrivals)
   uint64_t* bar_drain = bar_ph + 2;          // all MMAs of the CTA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_drain + 1);
+  // K/V tile records written by the producer (tile j at entry j % kMetaSlots; see tile_record)
+  volatile uint32_t* tile_meta = reinterpret_cast<volatile uint32_t*>(bars + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -472,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
   const int fa = text_rows ? p.T : r0 / p.P;
   const int fb = text_rows ? p.T : (r1 - 1) / p.P;
   const bool has1 = r0 + kBM < r1;  // the second query tile has rows
+  const bool pack = p.pack && fa == fb && !text_rows;  // every row of the block attends every run
   uint32_t* map_a = reinterpret_cast<uint32_t*>(smem + Cf::kOffMap);
   uint32_t* map_b = map_a + kMapWords;
   {
@@ -512,6 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       mbar_init(bar_ph + i, 4 * 32);
     }
     mbar_init(bar_drain, 1);
+    for (int i = 0; i < kMetaSlots; ++i) tile_meta[i] = 0xffff0000u;
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -553,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     int slot = 0;         // ring slot and phase of the next load
     uint32_t phase = 0;
     bool ok = true;
-    auto load = [&](const CUtensorMap* tm, int tok) {
+    auto load = [&](const CUtensorMap* tm, const CUtensorMap* tm8, int tok, int n_a, int tok_b) {
       if (!__all_sync(0xffffffffu, wait_bounded(bar_empty + slot, phase ^ 1, w))) {
         ok = false;
         return;
@@ -561,9 +624,20 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       if (elect_one()) {
         mbar_arrive_expect_tx(bar_full + slot, Cf::kTileBytes);
         uint8_t* dst = sRing + slot * Cf::kTileBytes;
+        if (tok_b == 0) {
 #pragma unroll
-        for (int c = 0; c < Cf::kChunks; ++c)
-          tma_load_3d(dst + c * kChunkBytes, tm, bar_full + slot, col0 + c * 64, tok, b);
+          for (int c = 0; c < Cf::kChunks; ++c)
+            tma_load_3d(dst + c * kChunkBytes, tm, bar_full + slot, col0 + c * 64, tok, b);
+        } else {
+          // a tile across two runs: rows [0, n_a) from tok, rows [n_a, 128) from tok_b, in 8-row boxes
+          // (1024 bytes of a 64-column chunk each, so every box lands on a swizzle-atom boundary)
+          const int ga = n_a >> 3;
+#pragma unroll
+          for (int c = 0; c < Cf::kChunks; ++c)
+            for (int g = 0; g < kBN / 8; ++g)
+              tma_load_3d(dst + c * kChunkBytes + g * 1024, tm8, bar_full + slot, col0 + c * 64,
+                          g < ga ? tok + 8 * g : tok_b + 8 * (g - ga), b);
+        }
       }
       __syncwarp();
       ++issued;
@@ -574,10 +648,25 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     };
     // consumption order of the MMA warp: K0, V0, K1, V1, ...
     FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
+    walk.pack = pack;
     int tok, nv, tmask;
-    while (ok && walk.next(tok, nv, tmask)) {
-      load(&p.tm_k, tok);
-      if (ok) load(&p.tm_v, tok);
+    bool have = walk.next(tok, nv, tmask);
+    int n_a = walk.n_a, tok_b = walk.n_a < nv ? walk.tok_b : 0;
+    if (!have && lane == 0) tile_meta[0] = tile_record(0, 0, 0, true);  // no tile at all
+    for (int j = 0; ok && have; ++j) {
+      int tok_n, nv_n, tmask_n;
+      const bool more = walk.next(tok_n, nv_n, tmask_n);
+      const int n_a_n = walk.n_a, tok_b_n = walk.n_a < nv_n ? walk.tok_b : 0;
+      if (lane == 0) tile_meta[j % kMetaSlots] = tile_record(j, nv, tmask, !more);
+      __syncwarp();  // the record is written before the loads' barrier arrivals
+      load(&p.tm_k, &p.tm_k8, tok, n_a, tok_b);
+      if (ok) load(&p.tm_v, &p.tm_v8, tok, n_a, tok_b);
+      n_a = n_a_n;
+      tok_b = tok_b_n;
+      tok = tok_n;
+      nv = nv_n;
+      tmask = tmask_n;
+      have = more;
     }
     if (!ok) {
       // stopped early: let every copy still in flight land before the CTA exits
@@ -640,10 +729,10 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       }
     };
     bool ok = wait_all(bar_q, 0);
-    FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
-    int tok, nv, tmask;
-    if (ok && walk.next(tok, nv, tmask)) {
-      int n_cur = (nv + 15) & ~15;
+    uint32_t rec = 0;
+    if (ok) ok = __all_sync(0xffffffffu, read_record(tile_meta, 0, w, rec));
+    if (ok && rec_nv(rec) > 0) {
+      int n_cur = (rec_nv(rec) + 15) & ~15;
       int k0;
       uint32_t k0p;
       take(k0, k0p);
@@ -663,9 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         __syncwarp();
       }
       for (int j = 0; ok; ++j) {
-        int tok_n, nv_n, tmask_n;
-        const bool has_next = walk.next(tok_n, nv_n, tmask_n);
-        const int n_next = (nv_n + 15) & ~15;
+        const bool has_next = !rec_last(rec);
+        int n_next = 0;
         int vi;
         uint32_t vph;
         take(vi, vph);
@@ -690,6 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
             ok = false;
             break;
           }
+          // the next tile's record was written before its K load was armed
+          rec = tile_meta[(j + 1) % kMetaSlots];
+          n_next = (rec_nv(rec) + 15) & ~15;
         }
         if (!wait_all(bar_p + 0, j & 1)) {
           ok = false;
@@ -759,9 +850,12 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
       int j = 0;
       const int row = r0 + qi * kBM + r;  // query row in the frame-major sequence
       const int rbit = (row / p.P == fa) ? 1 : 2;
-      FrameWalk walk(map_a, map_b, p.T, p.P, p.ntext);
-      int tok, nv, tmask;
-      while (walk.next(tok, nv, tmask)) {
+      for (;;) {
+        uint32_t rec;
+        ok = __all_sync(0xffffffffu, read_record(tile_meta, j, w, rec));
+        if (!ok) break;
+        const int nv = rec_nv(rec), tmask = rec_mask(rec);
+        if (nv == 0) break;  // no tile at all
         ok = __all_sync(0xffffffffu, wait_bounded(bar_s + qi, j & 1, w));
         if (!ok) break;
         tc_fence_after();
@@ -772,6 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         tc_fence_before();
         mbar_arrive(bar_p + qi);
         ++j;
+        if (rec_last(rec)) break;
       }
       // j == 0: the block walked no tile at all (its frames have no valid list entry); O in TMEM was never
       // written, and the rows get zeros

@@ -98,6 +98,9 @@ def test_negative_control_wrong_step_fails(gpu_lib):
     (7, 1, 2, 64, 1, 3, 1, 4),        # one token per frame
     (4, 2, 1, 128, 3, 2, 2, 1),       # two tokens per frame, batch 3
     (9, 130, 1, 128, 1, 1, 1, 0),     # C = W = 1: every frame attends only itself
+    (12, 520, 2, 128, 1, 6, 2, 5),    # P % 8 == 0: tiles span two runs (8 tokens of one, 120 of the next)
+    (12, 40, 2, 64, 2, 6, 2, 7),      # P % 8 == 0, frames shorter than a tile: packed tiles stay partial
+    (9, 1560, 1, 128, 1, 5, 2, 3),    # the 24-token frame tails packed with the next run
 ])
 def test_ragged_shapes_full_parity(gpu_lib, T, P, H, d, B, C, W, s):
     q, k, v = make(T, P, H, d, B=B, seed=T * 1000 + P)
