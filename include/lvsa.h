@@ -16,9 +16,11 @@
  *  - Every function returns an lvsa_status; nothing is thrown, nothing aborts.
  *  - Arguments are validated before any CUDA call or launch; on an error return
  *    no output has been written and nothing was launched.
- *  - The library never allocates device memory and never frees caller memory:
- *    the caller owns every buffer it passes (lvsa_ipc_import maps another
- *    process's buffer; lvsa_ipc_release unmaps it).
+ *  - The library never allocates device memory at run time and never frees
+ *    caller memory: the caller owns every buffer it passes (lvsa_ipc_import
+ *    maps another process's buffer; lvsa_ipc_release unmaps it).  The one
+ *    static device array of lvsa_attention_host_static is part of the loaded
+ *    module.
  *  - Thread safety: lvsa_build_frame_lists is pure; lvsa_attention and
  *    lvsa_attention_host may be called from several host threads.
  */
