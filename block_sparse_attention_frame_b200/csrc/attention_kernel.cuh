@@ -164,8 +164,9 @@ __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, long 
 // frame lists are held as bitmaps over [0, T) (so list order and duplicates do not
 // matter).  The walk visits the union in ascending frame order as runs of
 // consecutive frames with the same membership (bit 0: attended by fa, bit 1: by
-// fb); a run is one contiguous token range, cut into tiles of at most 128 tokens.
-// Every role of the CTA walks the same sequence.
+// fb); a run is one contiguous token range, cut into tiles of at most 128 tokens
+// (in a packed walk a tile may take the end of one run and the start of the next).
+// Only the TMA producer walks; the other roles read the tile records it publishes.
 struct FrameWalk {
   const uint32_t* ma;
   const uint32_t* mb;
@@ -682,7 +683,8 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
     // runs the schedule (descriptors stay warp-uniform); one elected lane issues each group of MMAs and
     // the commits that follow it.  The issuer shares a sub-partition with a softmax warp of each
     // warpgroup, so its instruction count sits on the P hand-off chain: descriptors are built as 32-bit
-    // low words, and there is one elected block per group rather than per MMA.
+    // low words, there is one elected block per group rather than per MMA, and the tile sequence comes
+    // from the producer's records instead of a walk of the lists.
     const uint32_t sq = smem_u32(sQ);
     const uint32_t sr = smem_u32(sRing);
     const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
