@@ -224,12 +224,11 @@ lvsa_status lvsa_attention_host(const void* q_host, const void* k_host, const vo
  *   LVSA_ERR_INVALID_ARG before anything is copied or launched.
  * Behaviour: asynchronous on `stream`; synchronise it before reading out_host.
  *   The first call on a device looks up the array's device address (one
- *   cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.  Every call on a device shares the one array,
- *   which keeps the previous call's contents (each call overwrites what it
- *   reads before reading it): calls whose work overlaps on the GPU (other
- *   streams, other host threads) race on it -- serialise them, e.g. on one
- *   stream.  Errors as lvsa_attention.
+ *   cudaGetSymbolAddress, with that device current).  Every call on a device
+ *   shares the one array, which keeps the previous call's contents (each call
+ *   overwrites what it reads before reading it): calls whose work overlaps on
+ *   the GPU (other streams, other host threads) race on it -- serialise them,
+ *   e.g. on one stream.  Errors as lvsa_attention.
  */
 lvsa_status lvsa_attention_host_static(const void* q_host, const void* k_host, const void* v_host,
                                        const int32_t* lists_host, int L, int T, int tokens_per_frame,
