@@ -296,12 +296,17 @@ def test_blocks_with_no_listed_frame_write_zeros(gpu_lib, T, P, d):
     assert_close(got[:, rows], ref, "other frames")
 
 
-def run_host_path(lib, q, k, v, lists_np, P, heads_per_band=0, scale=0.0):
-    """The host-buffer entry point: CPU tensors in, CPU tensor out, staging buffers on the GPU."""
+def run_host_path(lib, q, k, v, lists_np, P, heads_per_band=0, scale=0.0, stale=None):
+    """The host-buffer entry point: CPU tensors in, CPU tensor out, staging buffers on the GPU.  `stale`:
+    a value the staging buffers hold before the call (a row the kernel reads but the call did not upload
+    would leak it into the output)."""
     qh, kh, vh = (x.cpu().contiguous().pin_memory() for x in (q, k, v))
     lh = torch.from_numpy(np.ascontiguousarray(lists_np, dtype=np.int32))
     oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
     qd, kd, vd, od = (torch.empty(qh.shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    if stale is not None:
+        for x in (qd, kd, vd, od):
+            x.fill_(stale)
     ld = torch.empty(lh.shape, dtype=torch.int32, device="cuda")
     lib.lvsa_attention_host(qh, kh, vh, lh, P, oh, qd, kd, vd, ld, od, scale=scale, heads_per_band=heads_per_band)
     torch.cuda.synchronize()
@@ -322,11 +327,31 @@ def test_host_buffer_path_equals_device_path(gpu_lib, T, P, H, d, B, C, W, s, hb
     q, k, v = make(T, P, H, d, B=B, seed=11)
     lists = gpu_lib.lvsa_build_frame_lists(T, C, W, s)
     dev_out = run_kernel(gpu_lib, q, k, v, lists, P).cpu()
-    host_out = run_host_path(gpu_lib, q, k, v, lists, P, heads_per_band=hb)
+    # staging buffers full of NaN: every row the kernel reads must have been uploaded by the call
+    host_out = run_host_path(gpu_lib, q, k, v, lists, P, heads_per_band=hb, stale=float("nan"))
     # same kernel on the same bf16 inputs, one band of heads at a time: identical bits
     assert torch.equal(host_out.view(torch.int16), dev_out.view(torch.int16))
     ref = OA.sparse_attention(*host(q, k, v), OL.frame_lists(T, C, W, s), P)
     assert_close(host_out.float().numpy(), ref, "host-buffer path")
+
+
+@pytest.mark.parametrize("H,hb", [(3, 1), (2, 2)])
+def test_host_buffer_path_hand_made_lists(gpu_lib, H, hb):
+    """Lists made by hand (unsorted, a repeated entry, frames almost nobody lists, runs ending inside a
+    tile), staging buffers full of NaN: every row the kernel reads comes from the call's own uploads, and the
+    result is the device call's, bit for bit."""
+    T, P, d = 12, 520, 128
+    rows = []
+    for t in range(T):
+        rows.append([(t + 5) % T, t, 9 if t < 6 else 2, t])  # frame 9 or 2 for every row; 10, 11 mostly unread
+    lists = np.array(rows, dtype=np.int32)
+    q, k, v = make(T, P, H, d, seed=31)
+    dev_out = run_kernel(gpu_lib, q, k, v, lists, P).cpu()
+    host_out = run_host_path(gpu_lib, q, k, v, lists, P, heads_per_band=hb, stale=float("nan"))
+    assert torch.isfinite(host_out.float()).all()
+    assert torch.equal(host_out.view(torch.int16), dev_out.view(torch.int16))
+    ref = OA.sparse_attention(*host(q, k, v), [sorted(set(r)) for r in rows], P)
+    assert_close(host_out.float().numpy(), ref, "host-buffer path, hand-made lists")
 
 
 def test_host_buffer_path_full_size_heads(gpu_lib):
@@ -440,3 +465,38 @@ def test_cuda_graph_capture_and_replay(gpu_lib):
         torch.cuda.synchronize()
         assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
         assert torch.equal(oh.view(torch.int16), eager.cpu().view(torch.int16))
+
+
+def test_captured_host_call_follows_the_lists_at_replay(gpu_lib):
+    """A captured host-buffer call reads the host lists at replay: captured with the lists of step 3,
+    replayed after the host buffer was given those of step 4 (and the staging buffers filled with NaN), it
+    gives the eager result for step 4, bit for bit -- one graph serves every denoising step."""
+    T, P, H, d = 10, 300, 2, 128
+    q, k, v = make(T, P, H, d, seed=43)
+    qh, kh, vh = (x.cpu().contiguous().pin_memory() for x in (q, k, v))
+    lh = torch.from_numpy(gpu_lib.lvsa_build_frame_lists(T, 5, 2, 3)).pin_memory()
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    stage = [torch.empty_like(q) for _ in range(4)]
+    ld = torch.empty(lh.shape, dtype=torch.int32, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # first-call setup outside the capture
+        gpu_lib.lvsa_attention_host(qh, kh, vh, lh, P, oh, stage[0], stage[1], stage[2], ld, stage[3],
+                                    heads_per_band=1)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gpu_lib.lvsa_attention_host(qh, kh, vh, lh, P, oh, stage[0], stage[1], stage[2], ld, stage[3],
+                                    heads_per_band=1)
+    lists4 = gpu_lib.lvsa_build_frame_lists(T, 5, 2, 4)
+    assert not np.array_equal(lists4, lh.numpy())
+    lh.copy_(torch.from_numpy(lists4))
+    for x in stage:
+        x.fill_(float("nan"))
+    oh.zero_()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    eager = run_kernel(gpu_lib, q, k, v, lists4, P).cpu()
+    assert torch.equal(oh.view(torch.int16), eager.view(torch.int16))
