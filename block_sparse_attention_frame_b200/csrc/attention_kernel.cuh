@@ -632,12 +632,15 @@ __global__ void __launch_bounds__(kThreads, 1) lvsa_attention_kernel(const __gri
         } else {
           // a tile across two runs: rows [0, n_a) from tok, rows [n_a, 128) from tok_b, in 8-row boxes
           // (1024 bytes of a 64-column chunk each, so every box lands on a swizzle-atom boundary)
+          // (the box loop stays rolled: unrolled, its 32 coordinates spill the 56 registers of this warp)
           const int ga = n_a >> 3;
+#pragma unroll 1
+          for (int g = 0; g < kBN / 8; ++g) {
+            const int row = g < ga ? tok + 8 * g : tok_b + 8 * (g - ga);
 #pragma unroll
-          for (int c = 0; c < Cf::kChunks; ++c)
-            for (int g = 0; g < kBN / 8; ++g)
-              tma_load_3d(dst + c * kChunkBytes + g * 1024, tm8, bar_full + slot, col0 + c * 64,
-                          g < ga ? tok + 8 * g : tok_b + 8 * (g - ga), b);
+            for (int c = 0; c < Cf::kChunks; ++c)
+              tma_load_3d(dst + c * kChunkBytes + g * 1024, tm8, bar_full + slot, col0 + c * 64, row, b);
+          }
         }
       }
       __syncwarp();
