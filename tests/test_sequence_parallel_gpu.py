@@ -140,6 +140,16 @@ for step in (0, 3, 4):
     ref = lvsa.lvsa_attention(q, k, v, lists, P)
     torch.cuda.synchronize()
     ok = ok and torch.equal(out.view(torch.int16), ref[:, a:b].contiguous().view(torch.int16))
+# the same call on host buffers: this rank's range in and out
+qh, kh, vh = (x[:, a:b].cpu().contiguous().pin_memory() for x in (q, k, v))
+for step in (1, 4):
+    lists_np = lvsa.lvsa_build_frame_lists(T, 5, 3, step)
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    sp.host_call(qh, kh, vh, torch.from_numpy(lists_np).pin_memory(), oh)
+    torch.cuda.synchronize()
+    ref = lvsa.lvsa_attention(q, k, v, torch.from_numpy(lists_np).cuda(), P)
+    torch.cuda.synchronize()
+    ok = ok and torch.equal(oh.view(torch.int16), ref[:, a:b].cpu().contiguous().view(torch.int16))
 status = lvsa.lvsa_get_device_status(clear=True)
 sp.close()
 dist.destroy_process_group()
@@ -153,8 +163,9 @@ print("RESULT", rank, int(ok), status, flush=True)
 ])
 def test_processes_share_one_gpu_through_ipc(tmp_path, gpu_lib, world, heads, chunks):
     """Ranks as processes on one GPU: each maps the others' buffers (lvsa_ipc_import), gathers its heads from
-    them, and stores its output rows into them; each rank's output equals its rows of the single call.  Host
-    barriers order the ranks; no kernel waits on another process."""
+    them, and stores its output rows into them; each rank's output equals its rows of the single call, on
+    device buffers and through host_call on host buffers.  Host barriers order the ranks; no kernel waits on
+    another process."""
     port = _free_port()
     script = tmp_path / "worker.py"
     script.write_text(WORKER.format(root=ROOT, heads=heads, chunks=chunks))
