@@ -204,3 +204,40 @@ def test_attention_joint_argument_validation_without_gpu(lib):
     assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
     assert call() in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
     assert call(text=0) in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
+
+
+def test_host_static_argument_validation_without_gpu(lib):
+    """The allocation-free call validates everything, the size limit included, before any CUDA call."""
+    A = 1 << 24
+    M = 1 << 20
+    good = dict(q=A, k=A + M, v=A + 2 * M, lists=A + 3 * M, L=4, T=8, P=64, H=2, d=64, B=1, scale=0.0,
+                out=A + 4 * M)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return lib.lvsa_attention_host_static_raw(a["q"], a["k"], a["v"], a["lists"], a["L"], a["T"], a["P"],
+                                                  a["H"], a["d"], a["B"], a["scale"], a["out"], 0)
+
+    INV = lib.LVSA_ERR_INVALID_ARG
+    for name in ("q", "k", "v", "lists", "out"):
+        assert call(**{name: 0}) == INV, name
+    assert call(L=0) == INV
+    assert call(L=9) == INV
+    assert call(T=0) == INV
+    assert call(P=0) == INV
+    assert call(H=0) == INV
+    assert call(B=0) == INV
+    assert call(scale=float("nan")) == INV
+    assert call(d=96) == lib.LVSA_ERR_UNSUPPORTED
+    assert call(out=A + 64) == INV       # output overlaps q (each tensor is 128 KB here)
+    assert call(lists=A + 4 * M + 64) == INV   # lists inside the output
+    # Q, K, V and the output (each rounded up to 256 bytes) plus the lists must fit in the static array
+    n = lib.LVSA_STATIC_SCRATCH_BYTES
+    big = dict(q=A, k=A + n, v=A + 2 * n, lists=A + 3 * n, out=A + 4 * n, d=128, H=1, L=7)
+    assert call(T=32, P=2048, **big) == INV           # 4 x 16 MiB: nothing left for the lists
+    assert call(**dict(big, L=1), T=1, P=1 << 20) == INV   # one tensor alone beyond a quarter of the array
+    from conftest import cuda_available
+
+    if not cuda_available():
+        # the largest of these shapes that fits passes validation and stops at the device check
+        assert call(T=31, P=2048, **big) in (lib.LVSA_ERR_CUDA, lib.LVSA_ERR_UNSUPPORTED)
